@@ -1,0 +1,610 @@
+#!/usr/bin/env python
+"""Throughput of the Top-k + error-feedback compress on B200.
+
+Default workload: one error-feedback step on the ResNet-50-sized flat fp32
+gradient (n = 25,557,032, 90% Laplace(0, 1e-3) + 10% 1e-2 * Student-t(3) at
+random positions) with k = 25,557 (density 0.1%), lr = 0.1, the residual
+carried from step to step.  A "step" is one topk_ef_compress call: the fused
+accumulate pass, the threshold resolution and the ordered compaction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Prints ONE JSON line (rank 0).  value = algorithmic GB/s of the whole job:
+(12 B per element + 8 B per emitted pair) x elements of all ranks / device
+time, device time = sum over the K steps of CUDA-event intervals around each
+call on the launching stream, max over ranks.  L2 is flushed (256 MiB write)
+between steps, outside the timed intervals.  Multi-GPU: every rank
+compresses its own gradient (data-parallel replicas, no collective on the
+data path); torch.distributed is used only for the barrier and the max.
+
+--impl reference times the CPU oracle (oracle/, single thread) on a bounded
+sample of the same workload and prints the same line with "impl":
+"reference"; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import datagen  # noqa: E402
+
+METRIC = "Top-k+EF compress GB/s & elems/s at n=25.6M, density 0.1% (% of HBM peak)"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+LR = np.float32(0.1)
+POOL = 4          # distinct gradients cycled through the steps
+KERNEL_SOURCES = ["error_feedback_b200/csrc/kernels_compress.cuh",
+                  "error_feedback_b200/csrc/common.cuh"]
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def reduce_max(x: float, device=None) -> float:
+    """Max of x over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def sources_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch(kernel: str, n: int):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    summary, scaled to n elements; None if absent or the kernel changed."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if t.get("src_sha256") != sources_sha():
+        return None
+    return float(t["dram_bytes"]) * n / float(t["n"])
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, torch_dev: int, period_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = f"{type(e).__name__}: {e}"
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((mhz, int(rs)))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": self.err or "no samples"}
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [v for k, v in names.items() if mask & k and v != "gpu_idle"]
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workloads
+
+class FlatCompress:
+    """One EF step of topk_ef_compress on a flat gradient."""
+
+    def __init__(self, name, n, k, make_grad, label):
+        self.name, self.n, self.k, self.make_grad, self.label = name, n, k, make_grad, label
+        self.bytes_per_step = 12 * n + 8 * k
+        self.elems_per_step = n
+        self.dominant = "stream_kernel"
+        self.dominant_bytes = 12 * n     # read grad + read residual + write residual
+
+    def config(self):
+        return {"workload": self.label, "n": self.n, "k": self.k, "lr": float(LR),
+                "l2": "flushed between steps (256 MiB write); step inputs "
+                      f"{8 * self.n / 1e6:.0f} MB",
+                "parallelism": "replicas (one independent EF step per GPU)"}
+
+    def setup(self, rank, steps_needed):
+        import torch
+        import error_feedback_b200 as ef
+        self.ef = ef
+        npool = min(POOL, max(1, steps_needed))
+        self.host = [self.make_grad(100 * rank + s) for s in range(npool)]
+        self.dev = [torch.from_numpy(g).cuda() for g in self.host]
+        self.res = torch.zeros(self.n, dtype=torch.float32, device="cuda")
+        self.oi = torch.empty(max(self.k, 1), dtype=torch.int32, device="cuda")[:self.k]
+        self.ov = torch.empty(max(self.k, 1), dtype=torch.float32, device="cuda")[:self.k]
+        self.ws = torch.empty(ef.topk_ef_workspace_bytes(self.n, self.k), dtype=torch.uint8,
+                              device="cuda")
+        # host-buffer path: pinned gradient, device staging, pinned outputs
+        self.hpin = [torch.from_numpy(g).pin_memory() for g in self.host]
+        self.stage = torch.empty(self.n, dtype=torch.float32, device="cuda")
+        self.hoi = torch.empty(max(self.k, 1), dtype=torch.int32).pin_memory()[:self.k]
+        self.hov = torch.empty(max(self.k, 1), dtype=torch.float32).pin_memory()[:self.k]
+        self.h2d_bytes = 4 * self.n
+        self.d2h_bytes = 8 * self.k
+
+    def step(self, i):
+        self.ef.topk_ef_compress(self.dev[i % len(self.dev)], self.res, LR, self.k,
+                                 self.oi, self.ov, self.ws)
+
+    def e2e_step(self, i):
+        self.stage.copy_(self.hpin[i % len(self.hpin)], non_blocking=True)
+        self.ef.topk_ef_compress(self.stage, self.res, LR, self.k, self.oi, self.ov, self.ws)
+        self.hoi.copy_(self.oi, non_blocking=True)
+        self.hov.copy_(self.ov, non_blocking=True)
+
+    def status(self):
+        return self.ef.topk_ef_last_device_status(self.ws)
+
+    def path(self):
+        return self.ef.topk_ef_path_info(self.ws)
+
+    # CPU oracle on a bounded sample of the workload
+    def oracle_sample(self, budget_elems):
+        ns = int(min(self.n, max(1 << 16, budget_elems)))
+        ks = ns // max(1, round(self.n / max(self.k, 1))) if self.k else 0
+        ks = min(ks, ns)
+        g = self.make_grad(0)[:ns].copy()
+        return ns, ks, g
+
+
+class BatchedCompress:
+    """One EF step of topk_ef_compress_batched on the VGG-16 bucket."""
+
+    def __init__(self):
+        g, off, ks = datagen.vgg16_bucket(0)
+        self.offsets, self.ks = off, ks
+        self.n = int(off[-1])
+        self.k = int(ks.sum())
+        self.bytes_per_step = 12 * self.n + 8 * self.k
+        self.elems_per_step = self.n
+        self.dominant = "stream_kernel"
+        self.dominant_bytes = 12 * self.n
+        self._first = g
+
+    def config(self):
+        return {"workload": "vgg16_bucket: 16 VGG-16 weight tensors, Laplace(0, b_l), "
+                            "k_l = ceil(n_l/1000)", "n": self.n, "k": self.k, "lr": float(LR),
+                "l2": "flushed between steps (256 MiB write)",
+                "parallelism": "replicas (one independent EF step per GPU)"}
+
+    def setup(self, rank, steps_needed):
+        import torch
+        import error_feedback_b200 as ef
+        self.ef = ef
+        npool = min(2, max(1, steps_needed))
+        host = [self._first] + [datagen.vgg16_bucket(s)[0] for s in range(1, npool)]
+        self.dev = [torch.from_numpy(g).cuda() for g in host]
+        self.hpin = [torch.from_numpy(g).pin_memory() for g in host]
+        self.res = torch.zeros(self.n, dtype=torch.float32, device="cuda")
+        self.oi = torch.empty(self.k, dtype=torch.int32, device="cuda")
+        self.ov = torch.empty(self.k, dtype=torch.float32, device="cuda")
+        self.ws = torch.empty(ef.topk_ef_batched_workspace_bytes(self.offsets, self.ks),
+                              dtype=torch.uint8, device="cuda")
+        self.stage = torch.empty(self.n, dtype=torch.float32, device="cuda")
+        self.hoi = torch.empty(self.k, dtype=torch.int32).pin_memory()
+        self.hov = torch.empty(self.k, dtype=torch.float32).pin_memory()
+        self.h2d_bytes = 4 * self.n
+        self.d2h_bytes = 8 * self.k
+
+    def step(self, i):
+        self.ef.topk_ef_compress_batched(self.dev[i % len(self.dev)], self.res, self.offsets,
+                                         self.ks, LR, self.oi, self.ov, self.ws)
+
+    def e2e_step(self, i):
+        self.stage.copy_(self.hpin[i % len(self.hpin)], non_blocking=True)
+        self.ef.topk_ef_compress_batched(self.stage, self.res, self.offsets, self.ks, LR,
+                                         self.oi, self.ov, self.ws)
+        self.hoi.copy_(self.oi, non_blocking=True)
+        self.hov.copy_(self.ov, non_blocking=True)
+
+    def status(self):
+        return self.ef.topk_ef_last_device_status(self.ws)
+
+    def path(self):
+        return self.ef.topk_ef_path_info(self.ws)
+
+
+class Merge:
+    """One gTop-k tournament: P = 32 sets of k = 25,557 over n = 25,557,032."""
+
+    def __init__(self, P=32, k=25_557, n=datagen.RESNET50_N):
+        self.P, self.kin, self.k, self.nidx = P, k, k, n
+        rounds = (P - 1).bit_length()
+        # algorithmic bytes: every pair merge reads two sets and writes one
+        merges = P - 1
+        self.bytes_per_step = merges * 3 * 8 * k
+        self.elems_per_step = P * k
+        self.dominant = "merge_round_kernel"
+        self.dominant_bytes = None
+        self.rounds = rounds
+
+    def config(self):
+        return {"workload": f"gtopk_merge P={self.P} k={self.kin} n={self.nidx}",
+                "P": self.P, "k": self.k, "n": self.nidx,
+                "l2": "flushed between steps (256 MiB write); working set is L2-resident",
+                "parallelism": "P workers simulated on each GPU"}
+
+    def setup(self, rank, steps_needed):
+        import torch
+        import error_feedback_b200 as ef
+        self.ef = ef
+        idx, val = datagen.gtopk_sets(P=self.P, k=self.kin, n=self.nidx, step=rank)
+        self.di = torch.from_numpy(idx).cuda()
+        self.dv = torch.from_numpy(val).cuda()
+        self.hi = torch.from_numpy(idx).pin_memory()
+        self.hv = torch.from_numpy(val).pin_memory()
+        self.oi = torch.empty(self.k, dtype=torch.int32, device="cuda")
+        self.ov = torch.empty(self.k, dtype=torch.float32, device="cuda")
+        self.oc = torch.empty(1, dtype=torch.int32, device="cuda")
+        self.ws = torch.empty(ef.gtopk_merge_workspace_bytes(self.P, self.kin, self.k),
+                              dtype=torch.uint8, device="cuda")
+        self.si = torch.empty_like(self.di)
+        self.sv = torch.empty_like(self.dv)
+        self.hoi = torch.empty(self.k, dtype=torch.int32).pin_memory()
+        self.hov = torch.empty(self.k, dtype=torch.float32).pin_memory()
+        self.h2d_bytes = 8 * self.P * self.kin
+        self.d2h_bytes = 8 * self.k
+
+    def step(self, i):
+        self.ef.gtopk_merge(self.di, self.dv, self.k, self.nidx, self.oi, self.ov, self.oc,
+                            self.ws)
+
+    def e2e_step(self, i):
+        self.si.copy_(self.hi, non_blocking=True)
+        self.sv.copy_(self.hv, non_blocking=True)
+        self.ef.gtopk_merge(self.si, self.sv, self.k, self.nidx, self.oi, self.ov, self.oc,
+                            self.ws)
+        self.hoi.copy_(self.oi, non_blocking=True)
+        self.hov.copy_(self.ov, non_blocking=True)
+
+    def status(self):
+        return self.ef.topk_ef_last_device_status(self.ws)
+
+    def path(self):
+        return {}
+
+
+def make_workload(name):
+    n3 = datagen.RESNET50_N
+    if name in ("resnet50_mix", "resnet50_mix_0.1pct"):
+        return FlatCompress(name, n3, datagen.density_k(n3, 1e-3), datagen.resnet50_mix,
+                            "resnet50_mix: n=25,557,032, 90% Laplace(0,1e-3) + 10% "
+                            "1e-2*Student-t(3), k=25,557 (density 0.1%)")
+    if name == "resnet50_mix_1pct":
+        return FlatCompress(name, n3, datagen.density_k(n3, 1e-2), datagen.resnet50_mix,
+                            "resnet50_mix n=25,557,032 k=255,570 (density 1%)")
+    if name == "resnet50_mix_0.01pct":
+        return FlatCompress(name, n3, datagen.density_k(n3, 1e-4), datagen.resnet50_mix,
+                            "resnet50_mix n=25,557,032 k=2,555 (density 0.01%)")
+    if name == "flat_normal_1m":
+        return FlatCompress(name, 1 << 20, 1048, datagen.flat_normal,
+                            "flat_normal: n=1,048,576 N(0,1), k=1,048")
+    if name == "bf16_normal_1.5b":
+        return FlatCompress(name, datagen.LARGE_N, 1_500_000, datagen.bf16_normal,
+                            "bf16_normal: n=1.5e9, bf16-rounded N(0,1e-3), k=1.5e6")
+    if name == "vgg16_bucket":
+        return BatchedCompress()
+    if name == "gtopk_merge_p32":
+        return Merge()
+    raise SystemExit(f"unknown workload {name}")
+
+
+# --------------------------------------------------------------------- arms
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import error_feedback_b200 as ef
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    wl = make_workload(args.workload)
+    wl.setup(rank, args.steps + args.warmup)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    for w in range(args.warmup):
+        flush.fill_(float(w))
+        wl.step(w)
+    barrier()
+    st = wl.status()
+    if st != 0:
+        raise SystemExit(f"device status after warm-up: {ef.status_string(st)}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    ef.topk_ef_trace_enable(True)
+    barrier()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            wl.step(args.warmup + i)
+            ev[i][1].record(stream)
+        barrier()
+    trace = ef.topk_ef_trace_read()
+    ef.topk_ef_trace_enable(False)
+    st = wl.status()
+    if st != 0:
+        raise SystemExit(f"device status after timing: {ef.status_string(st)}")
+    path = wl.path()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = reduce_max(float(sum(step_ms)), "cuda")
+    units = world * args.steps
+    gbs = units * wl.bytes_per_step / (total_ms * 1e-3) / 1e9
+    eps = units * wl.elems_per_step / (total_ms * 1e-3)
+
+    # dominant kernel, timed by the library's events on the launch stream
+    dom = [ms for name, ms in trace if name == wl.dominant]
+    launches = len(trace)
+    roof = None
+    peak, peak_src = peaks()
+    if dom and wl.dominant_bytes:
+        avg = sum(dom) / len(dom)
+        ach = wl.dominant_bytes / (avg * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(ach, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+                "peak_source": f"{peak_src} (hbm_gbs, burst copy)",
+                "traffic": traffic_per_launch(wl.dominant, wl.n) if hasattr(wl, "n") else None,
+                "algorithmic_bytes_per_launch": wl.dominant_bytes,
+                "avg_launch_ms": round(avg, 5), "launches": len(dom)}
+    per_kernel = {}
+    for name, ms in trace:
+        d = per_kernel.setdefault(name, [0, 0.0])
+        d[0] += 1
+        d[1] += ms
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        ke = min(args.steps, 50)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(ke)]
+        for w in range(2):
+            wl.e2e_step(w)
+        barrier()
+        for i in range(ke):
+            ee[i][0].record(stream)
+            wl.e2e_step(i)
+            ee[i][1].record(stream)
+        barrier()
+        e_ms = reduce_max(float(sum(a.elapsed_time(b) for a, b in ee)), "cuda")
+        e2e = {"value": round(world * ke * wl.bytes_per_step / (e_ms * 1e-3) / 1e9, 2),
+               "unit": "GB/s", "h2d_bytes_per_step": wl.h2d_bytes,
+               "d2h_bytes_per_step": wl.d2h_bytes, "steps": ke,
+               "ms_per_step": round(e_ms / ke, 4)}
+
+    clocks = clk.summary()
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s",
+            "elems_per_s": round(eps, 1),
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": wl.config(),
+            "roofline": roof,
+            "hbm_frac_whole_step": round(gbs / world / peak, 4),
+            "gpu_launches": launches,
+            "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / v[0], 5)}
+                        for k, v in per_kernel.items()},
+            "path": path,
+            "e2e": e2e,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(wl, args)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def time_oracle(wl, steps, budget_elems):
+    """Run the oracle (full-sort back-end, one thread) for `steps` EF steps on
+    a bounded sample of the workload; returns (seconds, sample description,
+    bytes per step, elems per step)."""
+    import oracle
+    o = oracle.get()
+    if isinstance(wl, FlatCompress):
+        ns, ks, g = wl.oracle_sample(budget_elems)
+        res = np.zeros(ns, np.float32)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            o.compress(g, res, LR, ks, 0)
+        dt = time.perf_counter() - t0
+        return dt, f"{steps} EF steps on the first {ns} elements (k={ks})", 12 * ns + 8 * ks, ns
+    if isinstance(wl, BatchedCompress):
+        g, off, ks = datagen.vgg16_bucket(0)
+        res = np.zeros(g.size, np.float32)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            o.compress_batched(g, res, off, ks, LR, 0)
+        dt = time.perf_counter() - t0
+        return dt, f"{steps} EF steps on the full bucket", wl.bytes_per_step, wl.elems_per_step
+    if isinstance(wl, Merge):
+        idx, val = datagen.gtopk_sets(P=wl.P, k=wl.kin, n=wl.nidx)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            o.gtopk_merge(idx, val, wl.k, wl.nidx)
+        dt = time.perf_counter() - t0
+        return dt, f"{steps} full tournaments", wl.bytes_per_step, wl.elems_per_step
+    raise SystemExit("no oracle sample for this workload")
+
+
+def cpu_baseline(wl, args):
+    budget = wl.elems_per_step if isinstance(wl, FlatCompress) else None
+    if isinstance(wl, FlatCompress):
+        # about 15 s of single-thread work at ~5M elements/s
+        steps = max(1, min(3, int(75e6 // max(1, min(wl.n, 64 << 20)))))
+        dt, sample, bps, eps = time_oracle(wl, steps, min(wl.n, 64 << 20))
+    else:
+        steps = 1
+        dt, sample, bps, eps = time_oracle(wl, steps, budget)
+    return {"value": round(steps * bps / dt / 1e9, 4), "unit": "GB/s",
+            "elems_per_s": round(steps * eps / dt, 1), "cores": 1, "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 3)}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    wl = make_workload(args.workload)
+    # each step a bounded sample: the whole run stays near a minute
+    per_step_elems = int(max(1 << 16, min(getattr(wl, "n", 1 << 20),
+                                          300e6 / max(1, args.steps + args.warmup))))
+    if args.ref_elems:
+        per_step_elems = args.ref_elems
+    if isinstance(wl, FlatCompress):
+        ns, ks, g = wl.oracle_sample(per_step_elems)
+        import oracle
+        o = oracle.get()
+        res = np.zeros(ns, np.float32)
+        for _ in range(args.warmup):
+            o.compress(g, res, LR, ks, 0)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            o.compress(g, res, LR, ks, 0)
+        dt = time.perf_counter() - t0
+        bps, eps = 12 * ns + 8 * ks, ns
+        sample = f"each step: one EF step on the first {ns} elements (k={ks})"
+    else:
+        dt, sample, bps, eps = time_oracle(wl, args.steps, None)
+    gbs = args.steps * bps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "elems_per_s": round(args.steps * eps / dt, 1),
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": wl.config(),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="resnet50_mix")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-elems", type=int, default=0,
+                    help="reference arm: elements per step (default: sized to ~1 min)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, _, _ = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+// Device helpers shared by the Top-k + error-feedback kernels.
+//
+// |x| order: key(x) = bits(x) & 0x7FFFFFFF compared as an unsigned integer.
+// This equals the order of |x| for every non-NaN value (-0 == +0) and puts
+// NaN above +Inf, so "the k entries of largest absolute value" ("A
+// Distributed Synchronous SGD Algorithm with Global Top-k Sparsification for
+// Low Bandwidth Networks", ABSTRACT) is a total order once ties go to the
+// lower index.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tke {
+
+constexpr uint32_t KEY_MASK = 0x7FFFFFFFu;
+constexpr uint32_t DEAD = 0xFFFFFFFFu;      // empty slot of a merged list
+constexpr uint32_t NO_KEY = 0xFFFFFFFFu;    // threshold above every key
+
+// Radix digits of the 31-bit key: 11 + 10 + 10 bits.
+constexpr int D1_BITS = 11, D2_BITS = 10, D3_BITS = 10;
+constexpr int D1_BINS = 1 << D1_BITS;       // key >> 20
+constexpr int D2_BINS = 1 << D2_BITS;       // (key >> 10) & 1023
+constexpr int D3_BINS = 1 << D3_BITS;       // key & 1023
+constexpr int HIST_WORDS = D1_BINS + D1_BINS + D2_BINS + D3_BINS;  // per segment
+
+// Device status bits (ctrl.status).
+constexpr uint32_t ST_TIMEOUT = 1u;
+constexpr uint32_t ST_BAD_INPUT = 2u;
+constexpr uint32_t ST_INCONSISTENT = 4u;    // a count did not add up
+
+// Bounded waits: iterations of ~64 ns sleeps before a wait gives up.
+constexpr uint32_t SPIN_LIMIT = 1u << 22;
+
+// Control block at the start of every workspace.
+struct Ctrl {
+    uint32_t status;
+    uint32_t mode;          // compress: 0 prefilter path, 1 rescan fallback
+    uint32_t tile_ticket;   // dynamic tile counter of the streaming pass
+    uint32_t bar;           // grid barrier counter of the select kernel
+    uint64_t cand_total;    // candidates kept by the prefilter
+    uint64_t cap;           // candidate capacity
+    uint32_t kernels;       // kernels the call launched
+    uint32_t pad0;
+    uint32_t merge_bar[32]; // grid barrier counters, one per merge round
+    uint32_t pad1[6];
+};
+static_assert(sizeof(Ctrl) == 192, "Ctrl layout");
+
+__device__ __forceinline__ uint32_t key_of(float x) {
+    return __float_as_uint(x) & KEY_MASK;
+}
+
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Streaming 128-bit loads/stores (the data is touched once).
+__device__ __forceinline__ float4 ld_stream(const float4* p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(float4* p, float4 v) { __stcs(p, v); }
+
+__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
+__device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
+
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v) {
+    const uint32_t lane = lane_id();
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= (uint32_t)o) v += t;
+    }
+    return v;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// Block-wide exclusive scan.  s must hold 33 elements of shared memory.
+// Returns the exclusive prefix of v; *total receives the block sum.  Ends
+// with a __syncthreads so s may be reused right after.
+template <typename T>
+__device__ __forceinline__ T block_excl_scan(T v, T* s, T* total) {
+    const uint32_t lane = lane_id(), warp = warp_id();
+    const uint32_t nwarps = (blockDim.x + 31) >> 5;
+    T incl = warp_incl_scan(v);
+    if (lane == 31) s[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        T w = lane < nwarps ? s[lane] : T(0);
+        T wi = warp_incl_scan(w);
+        if (lane < nwarps) s[lane] = wi - w;
+        if (lane == 31) s[32] = wi;
+    }
+    __syncthreads();
+    T r = s[warp] + incl - v;
+    *total = s[32];
+    __syncthreads();
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ T block_sum(T v, T* s) {
+    T tot;
+    block_excl_scan(v, s, &tot);
+    return tot;
+}
+
+// Grid-wide barrier for a co-resident (cooperative) grid.  `counter` starts
+// at 0 for the launch and only grows; `epoch` counts the barriers this block
+// has passed.  Gives up after SPIN_LIMIT waits, records ST_TIMEOUT and
+// returns false: every block then leaves the kernel.
+__device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t& epoch,
+                                             uint32_t* status, int* s_flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        epoch += 1;
+        const uint32_t target = epoch * gridDim.x;
+        __threadfence();
+        atomicAdd(counter, 1u);
+        uint32_t it = 0;
+        int ok = 1;
+        while (ld_acquire_u32(counter) < target) {
+            if (++it > SPIN_LIMIT) {
+                atomicOr(status, ST_TIMEOUT);
+                ok = 0;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+        *s_flag = ok;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+// Find, in a histogram of nb bins (bin order = key order), the bin holding
+// the rem-th largest element (1-based) counting from the top bin down.
+// Executed by one full warp; every lane gets the result.
+//   bin   : the bin
+//   above : number of elements in bins above it
+//   cnt   : elements in the bin
+// Returns false when the histogram holds fewer than rem elements.
+__device__ __forceinline__ bool warp_find_bin(const uint32_t* h, int nb, uint32_t rem,
+                                              uint32_t& bin, uint32_t& above,
+                                              uint32_t& cnt) {
+    const uint32_t lane = lane_id();
+    const int per = nb >> 5;                       // bins per lane (power of two)
+    const int hi = nb - (int)lane * per;           // lane 0 owns the top bins
+    const int lo = hi - per;
+    uint32_t s = 0;
+    // rotated walk: lanes start at different banks
+    for (int i = 0; i < per; ++i) s += h[lo + ((i + (int)lane) & (per - 1))];
+    uint32_t incl = warp_incl_scan(s);
+    uint32_t excl = incl - s;
+    uint32_t hit = __ballot_sync(0xFFFFFFFFu, incl >= rem);
+    if (hit == 0) {
+        bin = 0;
+        above = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        cnt = 0;
+        return false;
+    }
+    const uint32_t src = __ffs(hit) - 1;
+    uint32_t rbin = 0, rabove = 0, rcnt = 0;
+    if (lane == src) {
+        uint32_t run = excl;
+        for (int b = hi - 1; b >= lo; --b) {
+            uint32_t c = h[b];
+            if (run + c >= rem) {
+                rbin = (uint32_t)b;
+                rabove = run;
+                rcnt = c;
+                break;
+            }
+            run += c;
+        }
+    }
+    bin = __shfl_sync(0xFFFFFFFFu, rbin, src);
+    above = __shfl_sync(0xFFFFFFFFu, rabove, src);
+    cnt = __shfl_sync(0xFFFFFFFFu, rcnt, src);
+    return true;
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) {
+    return (a + b - 1) / b;
+}
+
+}  // namespace tke

@@ -1,0 +1,447 @@
+// Segmented exact top-k selection and ordered emission.
+//
+// Input: a sequence of (index, value) positions split into segments (tensors
+// of a bucket, or the merged lists of the merge's pairs), each with its own
+// k.  For every segment the kernel finds the key T of its k-th element in
+// the order (|value| desc, index asc) by three radix digits of the 31-bit
+// key (11 + 10 + 10 bits), with the tie quota q = k - #{key > T}, and writes
+// the selected entries in index order:
+//     selected = {key > T} + the first q positions (in index order) with key == T
+// ("A Distributed Synchronous SGD Algorithm with Global Top-k Sparsification",
+// ABSTRACT: the k largest absolute values; lower index first among equal
+// magnitudes makes the set unique.)
+//
+// The grid is cooperative (all blocks resident): each block owns one
+// contiguous range of positions, histograms are summed in global memory and
+// separated by grid barriers, every block resolves the digits of the
+// segments it touches from those histograms, and the output offsets come
+// from per-block counts exchanged through a second barrier.
+#pragma once
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels_compress.cuh"
+
+namespace tke {
+
+constexpr int SEL_THREADS = 512;
+constexpr int SEG_MAX = 256;
+constexpr int EMIT_PER_THREAD = 4;
+constexpr int EMIT_TILE = SEL_THREADS * EMIT_PER_THREAD;
+
+struct Slot {
+    int32_t l_first, l_last;
+    uint32_t gt_first, eq_first, gt_last, eq_last;
+    uint32_t pad[2];
+};
+
+struct Resolved {
+    uint32_t none;     // k == 0: nothing selected
+    uint32_t prefix;   // decided high bits of T
+    uint32_t rem;      // rank still needed inside the prefix class
+    uint32_t T;        // the threshold key (after three digits)
+    uint32_t q;        // tie quota
+    uint32_t ok;
+};
+
+// ---------------------------------------------------------------- sources
+
+// Compress: candidates of the streaming pass, or the whole residual.
+struct CompressSrc {
+    float* resid;
+    int64_t N;
+    int32_t T;
+    const SegMeta* meta;
+    const int64_t* cand_start;   // [T+1]
+    const uint32_t* cand_idx;
+    const float* cand_val;
+    uint64_t cap;
+    uint32_t* hist;              // [T][HIST_WORDS]
+    int32_t* out_idx;
+    float* out_val;
+    int32_t force_dense;
+    int32_t dense;               // decided inside the kernel
+
+    __device__ int nseg() const { return T; }
+    __device__ int64_t seg_bound(int l) const { return dense ? (l < T ? meta[l].off : N) : cand_start[l]; }
+    __device__ uint32_t seg_k(int l) const { return meta[l].k; }
+    __device__ int first_digit() const { return dense ? 1 : 2; }
+    __device__ uint32_t* d1(int l) const { return hist + (size_t)l * HIST_WORDS + (dense ? D1_BINS : 0); }
+    __device__ uint32_t* d2(int l) const { return hist + (size_t)l * HIST_WORDS + 2 * D1_BINS; }
+    __device__ uint32_t* d3(int l) const { return hist + (size_t)l * HIST_WORDS + 2 * D1_BINS + D2_BINS; }
+    __device__ void load(int64_t pos, uint32_t& idx, float& val) const {
+        if (dense) { idx = (uint32_t)pos; val = resid[pos]; }
+        else { idx = cand_idx[pos]; val = cand_val[pos]; }
+    }
+    __device__ void emit(int l, uint32_t rank, uint32_t idx, float val) const {
+        const SegMeta& m = meta[l];
+        out_idx[m.out_base + rank] = (int32_t)((int64_t)idx - m.off);
+        out_val[m.out_base + rank] = val;
+        resid[idx] = 0.0f;
+    }
+    // Block-uniform decision: the prefilter holds the top-k of every tensor
+    // when each tensor kept at least k candidates and nothing was dropped.
+    __device__ void prepare(uint32_t* s_red, Ctrl* ctrl) {
+        const uint64_t total = (uint64_t)cand_start[T];
+        uint32_t bad = 0;
+        for (int l = threadIdx.x; l < T; l += blockDim.x)
+            bad |= (uint64_t)(cand_start[l + 1] - cand_start[l]) < (uint64_t)meta[l].k;
+        bad = block_sum(bad, s_red);
+        dense = (force_dense || total > cap || bad) ? 1 : 0;
+        if (blockIdx.x == 0 && threadIdx.x == 0) ctrl->mode = dense;
+    }
+    __device__ void finalize(const Resolved*) const {}
+};
+
+// Merge round: merged lists of the pairs (DEAD marks empty slots).
+struct MergeSrc {
+    const uint32_t* m_idx;
+    const float* m_val;
+    int64_t mcap;                // positions per segment
+    int32_t T;                   // segments (pairs)
+    const uint32_t* live;        // [T] entries in each merged list (or null)
+    uint32_t live_const;         // used when live is null
+    uint32_t kmax;
+    uint32_t* hist;              // [T][HIST_WORDS]
+    int32_t dense;               // always 0
+    int32_t d1_done;             // the merge kernel already built digit 1
+    int32_t final_out;
+    int32_t* out_idx;            // final: the caller's arrays
+    float* out_val;
+    int32_t* out_count;
+    int64_t out_k;
+    uint32_t* set_idx;           // otherwise: the sets buffer
+    float* set_val;
+    int64_t set_cap;
+    uint32_t* sizes;
+    int32_t pair_stride;         // 2^(r+1)
+    const uint32_t* bad_words;   // first select launch: input verdicts to fold
+    int32_t n_bad;
+
+    __device__ int nseg() const { return T; }
+    __device__ int64_t seg_bound(int l) const { return (int64_t)l * mcap; }
+    __device__ uint32_t seg_k(int l) const {
+        const uint32_t lv = live ? live[l] : live_const;
+        return lv < kmax ? lv : kmax;
+    }
+    __device__ int first_digit() const { return d1_done ? 2 : 1; }
+    __device__ uint32_t* d1(int l) const { return hist + (size_t)l * HIST_WORDS; }
+    __device__ uint32_t* d2(int l) const { return hist + (size_t)l * HIST_WORDS + 2 * D1_BINS; }
+    __device__ uint32_t* d3(int l) const { return hist + (size_t)l * HIST_WORDS + 2 * D1_BINS + D2_BINS; }
+    __device__ void load(int64_t pos, uint32_t& idx, float& val) const {
+        idx = m_idx[pos];
+        val = m_val[pos];
+    }
+    __device__ void emit(int l, uint32_t rank, uint32_t idx, float val) const {
+        if (final_out) {
+            out_idx[rank] = (int32_t)idx;
+            out_val[rank] = val;
+        } else {
+            const int64_t s = (int64_t)l * pair_stride * set_cap + rank;
+            set_idx[s] = idx;
+            set_val[s] = val;
+        }
+    }
+    __device__ void prepare(uint32_t*, Ctrl* ctrl) {
+        if (bad_words && blockIdx.x == 0 && threadIdx.x == 0) {
+            uint32_t any = 0;
+            for (int i = 0; i < n_bad; ++i) any |= bad_words[i];
+            if (any) atomicOr(&ctrl->status, ST_BAD_INPUT);
+        }
+    }
+    // Block 0: result lengths (and the padding of the caller's arrays).
+    __device__ void finalize_block0() const {
+        if (final_out) {
+            const uint32_t k0 = seg_k(0);
+            if (threadIdx.x == 0) *out_count = (int32_t)k0;
+            for (int64_t i = (int64_t)k0 + threadIdx.x; i < out_k; i += blockDim.x) {
+                out_idx[i] = -1;
+                out_val[i] = 0.0f;
+            }
+        } else {
+            for (int l = threadIdx.x; l < T; l += blockDim.x)
+                sizes[(int64_t)l * pair_stride] = seg_k(l);
+        }
+    }
+};
+
+struct SelCommon {
+    Ctrl* ctrl;
+    uint32_t* bar;
+    Slot* slots;
+};
+
+// ---------------------------------------------------------------- helpers
+
+template <class Src>
+__device__ __forceinline__ int seg_of_pos(const int64_t* s_seg, int T, int64_t p) {
+    // largest l < T with s_seg[l] <= p
+    int lo = 0, hi = T;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_seg[mid] <= p) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Resolve `upto` digits of segment l (block-wide; result in *res).
+template <class Src>
+__device__ void resolve(const Src& src, int l, int upto, uint32_t* s_stage, Resolved* res,
+                        uint32_t* status) {
+    const uint32_t k = src.seg_k(l);
+    if (k == 0 || upto == 0) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            res->none = (k == 0);
+            res->prefix = 0;
+            res->rem = k;
+            res->T = NO_KEY;
+            res->q = 0;
+            res->ok = 1;
+        }
+        __syncthreads();
+        return;
+    }
+    const uint32_t* h1 = src.d1(l);
+    const uint32_t* h2 = src.d2(l);
+    const uint32_t* h3 = src.d3(l);
+    for (int i = threadIdx.x; i < D1_BINS; i += blockDim.x) s_stage[i] = h1[i];
+    if (upto >= 2)
+        for (int i = threadIdx.x; i < D2_BINS; i += blockDim.x) s_stage[D1_BINS + i] = h2[i];
+    if (upto >= 3)
+        for (int i = threadIdx.x; i < D3_BINS; i += blockDim.x) s_stage[D1_BINS + D2_BINS + i] = h3[i];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        uint32_t rem = k, prefix = 0, bin, above, cnt;
+        bool ok = warp_find_bin(s_stage, D1_BINS, rem, bin, above, cnt);
+        rem -= above;
+        prefix = bin;
+        if (upto >= 2 && ok) {
+            ok = warp_find_bin(s_stage + D1_BINS, D2_BINS, rem, bin, above, cnt);
+            rem -= above;
+            prefix = (prefix << D2_BITS) | bin;
+        }
+        if (upto >= 3 && ok) {
+            ok = warp_find_bin(s_stage + D1_BINS + D2_BINS, D3_BINS, rem, bin, above, cnt);
+            rem -= above;
+            prefix = (prefix << D3_BITS) | bin;
+        }
+        if (threadIdx.x == 0) {
+            res->none = 0;
+            res->prefix = prefix;
+            res->rem = rem;
+            res->T = (upto >= 3) ? prefix : NO_KEY;
+            res->q = rem;
+            res->ok = ok;
+            if (!ok) atomicOr(status, ST_INCONSISTENT);
+        }
+    }
+    __syncthreads();
+}
+
+// digit d (1..3) of a key, and whether the key lies in the class decided by
+// the first d-1 digits (prefix)
+__device__ __forceinline__ uint32_t digit_of(uint32_t key, int d) {
+    return d == 1 ? (key >> 20) : (d == 2 ? ((key >> 10) & (D2_BINS - 1)) : (key & (D3_BINS - 1)));
+}
+__device__ __forceinline__ bool in_class(uint32_t key, int d, uint32_t prefix) {
+    return d == 1 ? true : (d == 2 ? ((key >> 20) == prefix) : ((key >> 10) == prefix));
+}
+
+// ---------------------------------------------------------------- kernel
+
+template <class Src>
+__global__ void __launch_bounds__(SEL_THREADS)
+select_kernel(Src src, SelCommon cm) {
+    __shared__ int64_t s_seg[SEG_MAX + 1];
+    __shared__ uint32_t s_stage[D1_BINS + D2_BINS + D3_BINS];
+    __shared__ uint32_t s_h1[D1_BINS];
+    __shared__ uint64_t s_scan[33];
+    __shared__ uint32_t s_red[33];
+    __shared__ Resolved s_res;
+    __shared__ int s_flag;
+    __shared__ uint32_t s_pre[4];
+
+    const int tid = threadIdx.x;
+    const int c = blockIdx.x;
+    const int G = gridDim.x;
+    uint32_t epoch = 0;
+    uint32_t* status = &cm.ctrl->status;
+
+    src.prepare(s_red, cm.ctrl);
+    const int T = src.nseg();
+    for (int l = tid; l <= T; l += blockDim.x) s_seg[l] = src.seg_bound(l);
+    __syncthreads();
+    const int64_t total = s_seg[T];
+
+    // contiguous range of this block (multiple of 4 positions)
+    int64_t S = ceil_div64(total, G);
+    S = (S + 3) & ~(int64_t)3;
+    const int64_t p0 = min((int64_t)c * S, total);
+    const int64_t p1 = min(p0 + S, total);
+    const bool has = p1 > p0;
+    const int l_first = has ? seg_of_pos<Src>(s_seg, T, p0) : 0;
+    const int l_last = has ? seg_of_pos<Src>(s_seg, T, p1 - 1) : -1;
+
+    // ---- digit passes
+    for (int d = src.first_digit(); d <= 3; ++d) {
+        for (int l = l_first; l <= l_last; ++l) {
+            const int64_t a = max(p0, s_seg[l]);
+            const int64_t b = min(p1, s_seg[l + 1]);
+            if (a >= b) continue;
+            resolve(src, l, d - 1, s_stage, &s_res, status);
+            if (s_res.none || !s_res.ok) continue;
+            const uint32_t prefix = s_res.prefix;
+            uint32_t* hd = d == 1 ? src.d1(l) : (d == 2 ? src.d2(l) : src.d3(l));
+            const bool use_smem = (d == 1) && (b - a) >= 4096;
+            if (use_smem) {
+                for (int i = tid; i < D1_BINS; i += blockDim.x) s_h1[i] = 0;
+                __syncthreads();
+            }
+            for (int64_t pos = a + tid; pos < b; pos += blockDim.x) {
+                uint32_t idx;
+                float val;
+                src.load(pos, idx, val);
+                if (idx == DEAD) continue;
+                const uint32_t key = key_of(val);
+                if (!in_class(key, d, prefix)) continue;
+                const uint32_t dg = digit_of(key, d);
+                if (use_smem) atomicAdd(&s_h1[dg], 1u);
+                else atomicAdd(&hd[dg], 1u);
+            }
+            if (use_smem) {
+                __syncthreads();
+                for (int i = tid; i < D1_BINS; i += blockDim.x)
+                    if (s_h1[i]) atomicAdd(&hd[i], s_h1[i]);
+                __syncthreads();
+            }
+        }
+        if (!grid_barrier(cm.bar, epoch, status, &s_flag)) return;
+    }
+
+    // ---- per-block counts of (key > T, key == T) in the first and last segment
+    uint32_t gtF = 0, eqF = 0, gtL = 0, eqL = 0;
+    for (int l = l_first; l <= l_last; ++l) {
+        if (l != l_first && l != l_last) continue;
+        const int64_t a = max(p0, s_seg[l]);
+        const int64_t b = min(p1, s_seg[l + 1]);
+        resolve(src, l, 3, s_stage, &s_res, status);
+        const uint32_t Tk = s_res.none ? NO_KEY : s_res.T;
+        uint32_t gt = 0, eq = 0;
+        for (int64_t pos = a + tid; pos < b; pos += blockDim.x) {
+            uint32_t idx;
+            float val;
+            src.load(pos, idx, val);
+            if (idx == DEAD) continue;
+            const uint32_t key = key_of(val);
+            gt += key > Tk && Tk != NO_KEY;
+            eq += key == Tk;
+        }
+        gt = block_sum(gt, s_red);
+        eq = block_sum(eq, s_red);
+        if (l == l_first) { gtF = gt; eqF = eq; }
+        if (l == l_last) { gtL = gt; eqL = eq; }
+    }
+    if (tid == 0) {
+        Slot sl;
+        sl.l_first = has ? l_first : 0x7FFFFFFF;
+        sl.l_last = has ? l_last : -1;
+        sl.gt_first = gtF;
+        sl.eq_first = eqF;
+        sl.gt_last = gtL;
+        sl.eq_last = eqL;
+        sl.pad[0] = sl.pad[1] = 0;
+        cm.slots[c] = sl;
+    }
+    if (c == 0) {
+        if constexpr (std::is_same<Src, MergeSrc>::value) src.finalize_block0();
+    }
+    if (!grid_barrier(cm.bar, epoch, status, &s_flag)) return;
+
+    // ---- emission
+    for (int l = l_first; l <= l_last; ++l) {
+        const int64_t a = max(p0, s_seg[l]);
+        const int64_t b = min(p1, s_seg[l + 1]);
+        if (a >= b) continue;
+        resolve(src, l, 3, s_stage, &s_res, status);
+        if (s_res.none) continue;
+        const uint32_t Tk = s_res.T;
+        const uint32_t q = s_res.q;
+        const uint32_t kseg = src.seg_k(l);
+        // counts of earlier blocks in this segment
+        if (tid < 32) {
+            uint32_t pg = 0, pe = 0;
+            if (l == l_first && a > s_seg[l]) {
+                int cc = c - 1;
+                for (;;) {
+                    const int j = cc - (int)lane_id();
+                    bool valid = j >= 0, match = false, cont = false;
+                    uint32_t g = 0, e = 0;
+                    if (valid) {
+                        const Slot sl = cm.slots[j];
+                        match = sl.l_last == l;
+                        cont = match && sl.l_first == l;
+                        g = sl.gt_last;
+                        e = sl.eq_last;
+                    }
+                    const uint32_t contm = __ballot_sync(0xFFFFFFFFu, cont);
+                    const uint32_t matchm = __ballot_sync(0xFFFFFFFFu, match);
+                    const uint32_t run = (contm == 0xFFFFFFFFu) ? 32u : (uint32_t)(__ffs(~contm) - 1);
+                    const bool take = lane_id() < run || (lane_id() == run && ((matchm >> run) & 1u));
+                    pg += warp_sum(take ? g : 0u);
+                    pe += warp_sum(take ? e : 0u);
+                    if (run < 32) break;
+                    cc -= 32;
+                }
+            }
+            if (tid == 0) {
+                s_pre[0] = pg;
+                s_pre[1] = pe;
+            }
+        }
+        __syncthreads();
+        uint32_t run_gt = s_pre[0], run_eq = s_pre[1];
+        __syncthreads();
+        for (int64_t base = a; base < b; base += EMIT_TILE) {
+            uint32_t idx[EMIT_PER_THREAD];
+            float val[EMIT_PER_THREAD];
+            uint32_t cls = 0;   // bit u: gt, bit 4+u: eq
+#pragma unroll
+            for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+                const int64_t pos = base + (int64_t)tid * EMIT_PER_THREAD + u;
+                idx[u] = DEAD;
+                val[u] = 0.f;
+                if (pos < b) src.load(pos, idx[u], val[u]);
+                if (idx[u] != DEAD) {
+                    const uint32_t key = key_of(val[u]);
+                    if (key > Tk) cls |= 1u << u;
+                    else if (key == Tk) cls |= 1u << (4 + u);
+                }
+            }
+            const uint64_t mine = ((uint64_t)__popc(cls & 0xFu) << 32) | (uint64_t)__popc(cls >> 4);
+            uint64_t tot;
+            const uint64_t ex = block_excl_scan(mine, s_scan, &tot);
+            uint32_t g = run_gt + (uint32_t)(ex >> 32);
+            uint32_t e = run_eq + (uint32_t)(ex & 0xFFFFFFFFu);
+#pragma unroll
+            for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+                if ((cls >> u) & 1u) {
+                    const uint32_t rank = g + (e < q ? e : q);
+                    if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
+                    ++g;
+                } else if ((cls >> (4 + u)) & 1u) {
+                    if (e < q) {
+                        const uint32_t rank = g + e;
+                        if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
+                    }
+                    ++e;
+                }
+            }
+            run_gt += (uint32_t)(tot >> 32);
+            run_eq += (uint32_t)(tot & 0xFFFFFFFFu);
+        }
+    }
+}
+
+}  // namespace tke

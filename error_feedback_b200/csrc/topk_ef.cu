@@ -1,0 +1,688 @@
+// Host side of the C ABI declared in include/topk_ef.h: argument checks,
+// workspace layout and the launch sequence of each call.
+//
+//   topk_ef_compress / _batched:  setup_kernel -> stream_kernel -> select_kernel
+//   gtopk_merge:                  merge_setup_kernel -> (merge_round_kernel ->
+//                                 select_kernel) per tournament round
+//
+// Every launch goes to the caller's stream; nothing is allocated and nothing
+// is synchronised except by the two status read-back calls.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "topk_ef.h"
+#include "common.cuh"
+#include "kernels_compress.cuh"
+#include "kernels_merge.cuh"
+#include "kernels_select.cuh"
+
+using namespace tke;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+std::atomic<int> g_test_flags{0};
+
+constexpr int64_t MAX_N = 2147483647LL;
+constexpr int64_t SMALL_N = 65536;     // tensors up to this size are not sampled
+constexpr int SLOT_MAX = 2048;         // select grid never exceeds this
+constexpr size_t ALIGN = 256;
+constexpr int MAX_MERGE_P = 2 * SEG_MAX;   // pairs per round <= SEG_MAX
+
+size_t align_up(size_t x, size_t a = ALIGN) { return (x + a - 1) / a * a; }
+
+int cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return TOPK_EF_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ tracing
+// When enabled, every kernel launch is bracketed by two CUDA events on the
+// call's stream; records accumulate until they are read back.
+
+constexpr int TRACE_MAX = 4096;
+
+struct Trace {
+    int on = 0;
+    int dev = -1;
+    int n = 0;
+    cudaEvent_t ev[2 * TRACE_MAX] = {};
+    const char* name[TRACE_MAX] = {};
+};
+Trace g_trace;
+std::mutex g_trace_mu;
+
+void trace_before(cudaStream_t st, const char* name) {
+    if (!g_trace.on || g_trace.n >= TRACE_MAX) return;
+    g_trace.name[g_trace.n] = name;
+    cudaEventRecord(g_trace.ev[2 * g_trace.n], st);
+}
+
+void trace_after(cudaStream_t st) {
+    if (!g_trace.on || g_trace.n >= TRACE_MAX) return;
+    cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st);
+    ++g_trace.n;
+}
+
+// ------------------------------------------------------------ device facts
+
+struct DevFacts {
+    int sms = 0;
+    int k1_blocks = 0;       // resident stream_kernel blocks per SM
+    int selc_blocks = 0;     // resident select_kernel<CompressSrc> blocks per SM
+    int selm_blocks = 0;     // resident select_kernel<MergeSrc> blocks per SM
+};
+
+std::mutex g_facts_mu;
+DevFacts g_facts[64];
+bool g_facts_ready[64];
+
+int device_facts(DevFacts* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return TOPK_EF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_facts_mu);
+    if (!g_facts_ready[dev]) {
+        DevFacts f;
+        if ((e = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.k1_blocks, stream_kernel<true>,
+                                                               K1_THREADS, 0)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                 &f.selc_blocks, select_kernel<CompressSrc>, SEL_THREADS, 0)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                 &f.selm_blocks, select_kernel<MergeSrc>, SEL_THREADS, 0)) != cudaSuccess)
+            return cuda_fail(e);
+        if (f.sms <= 0 || f.k1_blocks <= 0 || f.selc_blocks <= 0 || f.selm_blocks <= 0)
+            return TOPK_EF_ERR_CUDA;
+        g_facts[dev] = f;
+        g_facts_ready[dev] = true;
+    }
+    *out = g_facts[dev];
+    return TOPK_EF_OK;
+}
+
+// ------------------------------------------------------- compress planning
+
+// Per tensor: samples taken for the prefilter threshold, the rank of the
+// threshold among them, and the candidate capacity reserved for it.
+struct TensorPlan {
+    int64_t off, n, out_base;
+    uint32_t k, m, r;
+    int64_t cap;
+};
+
+TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
+    TensorPlan t;
+    t.off = off;
+    t.n = n;
+    t.out_base = out_base;
+    t.k = (uint32_t)k;
+    t.m = 0;
+    t.r = 0;
+    if (k == 0) {
+        t.cap = 0;
+    } else if (n <= SMALL_N) {
+        t.cap = n;
+    } else {
+        // Expected sample count above the k-th key: ks = k * m / n.  Aim the
+        // threshold at ks + 6 sqrt(ks) + 16 samples so that it is below the
+        // k-th key unless the sample is far from typical.
+        const double m = (double)SAMPLE_M;
+        const double ks = (double)k * m / (double)n;
+        const double r = std::ceil(ks + 6.0 * std::sqrt(ks) + 16.0);
+        if (r >= m) {
+            t.cap = n;
+        } else {
+            t.m = (uint32_t)SAMPLE_M;
+            t.r = (uint32_t)r;
+            const double e = 2.5 * r * (double)n / m + 4096.0;
+            t.cap = std::min<int64_t>(n, (int64_t)std::ceil(e));
+        }
+    }
+    return t;
+}
+
+// Workspace layout of one compress group (<= TCAP_LARGE tensors).
+struct CLayout {
+    size_t ctrl, meta, zero_begin, cand_start, hist, tile_status, zero_end, slots, cand_idx,
+        cand_val, total;
+    int64_t cap;
+    uint32_t num_tiles;
+};
+
+CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
+    CLayout L;
+    const size_t T = plans.size();
+    int64_t cap = 0;
+    for (const auto& p : plans) cap += p.cap;
+    L.cap = cap;
+    L.num_tiles = (uint32_t)ceil_div64(N, TILE);
+    size_t o = 0;
+    L.ctrl = o;
+    o = align_up(o + sizeof(Ctrl));
+    L.meta = o;
+    o = align_up(o + T * sizeof(SegMeta));
+    L.zero_begin = o;
+    L.cand_start = o;
+    o = align_up(o + (T + 1) * sizeof(int64_t));
+    L.hist = o;
+    o = align_up(o + T * HIST_WORDS * sizeof(uint32_t));
+    L.tile_status = o;
+    o = align_up(o + (size_t)L.num_tiles * sizeof(uint64_t));
+    L.zero_end = o;
+    L.slots = o;
+    o = align_up(o + SLOT_MAX * sizeof(Slot));
+    L.cand_idx = o;
+    o = align_up(o + (size_t)cap * sizeof(uint32_t));
+    L.cand_val = o;
+    o = align_up(o + (size_t)cap * sizeof(float));
+    L.total = o;
+    return L;
+}
+
+// Validated per-group description of a (batched) compress call.
+struct Group {
+    int32_t t0, t1;                 // tensors [t0, t1)
+    std::vector<TensorPlan> plans;  // offsets local to the group
+    int64_t base;                   // first element of the group in the bucket
+    int64_t N;                      // elements in the group
+};
+
+int make_groups(const int64_t* offsets, const int64_t* k, int32_t T, std::vector<Group>* out) {
+    if (!offsets || !k || T < 1) return TOPK_EF_ERR_INVALID_ARG;
+    if (offsets[0] != 0) return TOPK_EF_ERR_INVALID_ARG;
+    for (int32_t l = 0; l < T; ++l) {
+        const int64_t n = offsets[l + 1] - offsets[l];
+        if (n < 0 || k[l] < 0 || k[l] > n) return TOPK_EF_ERR_INVALID_ARG;
+    }
+    if (offsets[T] > MAX_N) return TOPK_EF_ERR_INVALID_ARG;
+    int64_t out_base = 0;
+    for (int32_t g0 = 0; g0 < T; g0 += TCAP_LARGE) {
+        Group g;
+        g.t0 = g0;
+        g.t1 = std::min<int32_t>(T, g0 + TCAP_LARGE);
+        g.base = offsets[g0];
+        g.N = offsets[g.t1] - g.base;
+        for (int32_t l = g.t0; l < g.t1; ++l) {
+            g.plans.push_back(plan_tensor(offsets[l] - g.base, offsets[l + 1] - offsets[l], k[l],
+                                          out_base));
+            out_base += k[l];
+        }
+        out->push_back(std::move(g));
+    }
+    return TOPK_EF_OK;
+}
+
+size_t groups_workspace(const std::vector<Group>& groups) {
+    size_t mx = 0;
+    for (const auto& g : groups) mx = std::max(mx, compress_layout(g.N, g.plans).total);
+    return mx;
+}
+
+template <int TCAP>
+cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float* grad,
+                         const float* resid, float lr, bool force_t0_zero, uint32_t kernels,
+                         cudaStream_t st) {
+    SetupParams<TCAP> p;
+    memset(&p, 0, sizeof(p));
+    const int T = (int)g.plans.size();
+    p.grad = grad;
+    p.resid = resid;
+    p.lr = lr;
+    p.T = T;
+    p.kernels = kernels;
+    p.cap = (uint64_t)L.cap;
+    p.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+    p.meta = reinterpret_cast<SegMeta*>(ws + L.meta);
+    p.zero_ptr = reinterpret_cast<uint4*>(ws + L.zero_begin);
+    p.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
+    int ns = 0;
+    for (int l = 0; l < T; ++l) {
+        const TensorPlan& t = g.plans[l];
+        p.off[l] = t.off;
+        p.out_base[l] = t.out_base;
+        p.k[l] = t.k;
+        p.m[l] = force_t0_zero ? 0u : t.m;
+        p.r[l] = t.r;
+        if (p.m[l]) p.sampled[ns++] = (uint16_t)l;
+    }
+    p.off[T] = g.N;
+    p.n_sampled = ns;
+    const uint64_t per_block = (uint64_t)ZERO_THREADS * 8;
+    const int nz = (int)std::max<uint64_t>(1, std::min<uint64_t>(148, (p.zero_vec4 + per_block - 1) / per_block));
+    setup_kernel<TCAP><<<ns + nz, SAMPLE_THREADS, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+int compress_group(const Group& g, const float* grad, float* resid, float lr, int32_t* out_idx,
+                   float* out_val, char* ws, cudaStream_t st, const DevFacts& f, int flags) {
+    const CLayout L = compress_layout(g.N, g.plans);
+    const int T = (int)g.plans.size();
+    const bool force_dense = (flags & 1) != 0;
+    const bool force_t0 = (flags & 2) != 0;
+    const uint32_t kernels = g.N > 0 ? 3u : 1u;
+    const float* gg = grad + g.base;
+    float* rg = resid + g.base;
+    trace_before(st, "setup_kernel");
+    cudaError_t e = T <= TCAP_SMALL
+                        ? launch_setup<TCAP_SMALL>(g, L, ws, gg, rg, lr, force_t0, kernels, st)
+                        : launch_setup<TCAP_LARGE>(g, L, ws, gg, rg, lr, force_t0, kernels, st);
+    trace_after(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (g.N == 0) return TOPK_EF_OK;
+
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+    StreamParams sp;
+    sp.grad = gg;
+    sp.resid = rg;
+    sp.lr = lr;
+    sp.T = T;
+    sp.N = g.N;
+    sp.num_tiles = L.num_tiles;
+    sp.meta = reinterpret_cast<const SegMeta*>(ws + L.meta);
+    sp.ctrl = ctrl;
+    sp.tile_status = reinterpret_cast<uint64_t*>(ws + L.tile_status);
+    sp.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
+    sp.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
+    sp.cap = (uint64_t)L.cap;
+    sp.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+    sp.cand_start = reinterpret_cast<int64_t*>(ws + L.cand_start);
+    const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
+    const int g1 = (int)std::min<int64_t>(L.num_tiles, (int64_t)f.sms * f.k1_blocks);
+    trace_before(st, "stream_kernel");
+    if (vec) stream_kernel<true><<<g1, K1_THREADS, 0, st>>>(sp);
+    else stream_kernel<false><<<g1, K1_THREADS, 0, st>>>(sp);
+    trace_after(st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+
+    CompressSrc src;
+    memset(&src, 0, sizeof(src));
+    src.resid = rg;
+    src.N = g.N;
+    src.T = T;
+    src.meta = sp.meta;
+    src.cand_start = sp.cand_start;
+    src.cand_idx = sp.cand_idx;
+    src.cand_val = sp.cand_val;
+    src.cap = sp.cap;
+    src.hist = sp.hist;
+    src.out_idx = out_idx;
+    src.out_val = out_val;
+    src.force_dense = force_dense ? 1 : 0;
+    src.dense = 0;
+    SelCommon cm;
+    cm.ctrl = ctrl;
+    cm.bar = &ctrl->bar;
+    cm.slots = reinterpret_cast<Slot*>(ws + L.slots);
+    const int G = std::min(SLOT_MAX, f.sms * f.selc_blocks);
+    void* args[] = {&src, &cm};
+    trace_before(st, "select_kernel<CompressSrc>");
+    e = cudaLaunchCooperativeKernel((const void*)select_kernel<CompressSrc>, dim3(G),
+                                    dim3(SEL_THREADS), args, 0, st);
+    trace_after(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return TOPK_EF_OK;
+}
+
+bool bad_fp32_ptr(const void* p) { return ((uintptr_t)p & 3u) != 0; }
+
+// --------------------------------------------------------- merge planning
+
+struct MLayout {
+    size_t ctrl, sizes, bad, zero_begin, hist, live, zero_end, slots, set_idx, set_val, m_idx,
+        m_val, total;
+    int64_t cap;
+    int rounds;
+    std::vector<int32_t> np;       // pairs per round
+    std::vector<int64_t> mcap;     // merged positions per pair per round
+    std::vector<int64_t> pbase;    // first pair-merge id of each round
+    int64_t merges;                // total pair merges
+    int64_t mmax;                  // merged positions buffer
+    uint32_t vblocks;
+};
+
+MLayout merge_layout(int32_t P, int64_t k_in, int64_t k) {
+    MLayout L;
+    L.cap = std::max<int64_t>(1, std::max<int64_t>(k_in, std::min<int64_t>(k, (int64_t)P * k_in)));
+    L.rounds = 0;
+    while ((1LL << L.rounds) < P) ++L.rounds;
+    L.merges = 0;
+    L.mmax = 0;
+    for (int r = 0; r < L.rounds; ++r) {
+        const int64_t step = 1LL << r;
+        const int32_t np = (int32_t)((P - step - 1) / (2 * step) + 1);
+        const int64_t bound = std::min<int64_t>(L.cap, k_in << std::min(r, 40));
+        const int64_t mc = 2 * std::max<int64_t>(bound, 1);
+        L.np.push_back(np);
+        L.mcap.push_back(mc);
+        L.pbase.push_back(L.merges);
+        L.merges += np;
+        L.mmax = std::max<int64_t>(L.mmax, (int64_t)np * mc);
+    }
+    const int64_t hsegs = std::max<int64_t>(1, L.merges);
+    const int64_t tot = (int64_t)P * k_in;
+    L.vblocks = tot > 0 ? (uint32_t)std::min<int64_t>(148, ceil_div64(tot, MZ_THREADS * 8)) : 0u;
+    size_t o = 0;
+    L.ctrl = o;
+    o = align_up(o + sizeof(Ctrl));
+    L.sizes = o;
+    o = align_up(o + (size_t)P * sizeof(uint32_t));
+    L.bad = o;
+    o = align_up(o + 148 * sizeof(uint32_t));
+    L.zero_begin = o;
+    L.hist = o;
+    o = align_up(o + (size_t)hsegs * HIST_WORDS * sizeof(uint32_t));
+    L.live = o;
+    o = align_up(o + (size_t)hsegs * sizeof(uint32_t));
+    L.zero_end = o;
+    L.slots = o;
+    o = align_up(o + SLOT_MAX * sizeof(Slot));
+    L.set_idx = o;
+    o = align_up(o + (size_t)P * L.cap * sizeof(uint32_t));
+    L.set_val = o;
+    o = align_up(o + (size_t)P * L.cap * sizeof(float));
+    L.m_idx = o;
+    o = align_up(o + (size_t)L.mmax * sizeof(uint32_t));
+    L.m_val = o;
+    o = align_up(o + (size_t)L.mmax * sizeof(float));
+    L.total = o;
+    return L;
+}
+
+int merge_args_ok(int32_t P, int64_t k_in, int64_t k, int64_t n) {
+    if (P < 1 || P > MAX_MERGE_P || k_in < 0 || k < 0 || n < 0 || n > MAX_N || k_in > n)
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (k > MAX_N || (int64_t)P * k_in > (int64_t)1 << 40) return TOPK_EF_ERR_INVALID_ARG;
+    return TOPK_EF_OK;
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+
+extern "C" {
+
+size_t topk_ef_workspace_bytes(int64_t n, int64_t k) {
+    if (n < 0 || k < 0 || k > n || n > MAX_N) return 0;
+    const int64_t offsets[2] = {0, n};
+    return topk_ef_batched_workspace_bytes(offsets, &k, 1);
+}
+
+size_t topk_ef_batched_workspace_bytes(const int64_t* offsets, const int64_t* k, int32_t T) {
+    std::vector<Group> groups;
+    if (make_groups(offsets, k, T, &groups) != TOPK_EF_OK) return 0;
+    return groups_workspace(groups);
+}
+
+int topk_ef_compress_batched(const float* grad, float* residual, const int64_t* offsets,
+                             const int64_t* k, int32_t T, float lr, int32_t* out_idx,
+                             float* out_val, void* ws, size_t ws_bytes, void* stream) {
+    std::vector<Group> groups;
+    int rc = make_groups(offsets, k, T, &groups);
+    if (rc != TOPK_EF_OK) return rc;
+    const int64_t N = offsets[T];
+    int64_t ktot = 0;
+    for (int32_t l = 0; l < T; ++l) ktot += k[l];
+    if (!ws) return TOPK_EF_ERR_INVALID_ARG;
+    if (N > 0 && (!grad || !residual || bad_fp32_ptr(grad) || bad_fp32_ptr(residual)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (ktot > 0 && (!out_idx || !out_val || bad_fp32_ptr(out_val) || bad_fp32_ptr(out_idx)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (((uintptr_t)ws % ALIGN) != 0) return TOPK_EF_ERR_INVALID_ARG;
+    if (ws_bytes < groups_workspace(groups)) return TOPK_EF_ERR_WORKSPACE;
+    DevFacts f;
+    if ((rc = device_facts(&f)) != TOPK_EF_OK) return rc;
+    const int flags = g_test_flags.load();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (const auto& g : groups) {
+        rc = compress_group(g, grad, residual, lr, out_idx, out_val, (char*)ws, st, f, flags);
+        if (rc != TOPK_EF_OK) return rc;
+    }
+    return TOPK_EF_OK;
+}
+
+int topk_ef_compress(const float* grad, float* residual, int64_t n, float lr, int64_t k,
+                     int32_t* out_idx, float* out_val, void* ws, size_t ws_bytes, void* stream) {
+    if (n < 0 || k < 0 || k > n || n > MAX_N) return TOPK_EF_ERR_INVALID_ARG;
+    const int64_t offsets[2] = {0, n};
+    return topk_ef_compress_batched(grad, residual, offsets, &k, 1, lr, out_idx, out_val, ws,
+                                    ws_bytes, stream);
+}
+
+size_t gtopk_merge_workspace_bytes(int32_t P, int64_t k_in, int64_t k) {
+    if (P < 1 || P > MAX_MERGE_P || k_in < 0 || k < 0) return 0;
+    return merge_layout(P, k_in, k).total;
+}
+
+int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k_in, int64_t k,
+                int64_t n, int32_t* out_idx, float* out_val, int32_t* out_count, void* ws,
+                size_t ws_bytes, void* stream) {
+    int rc = merge_args_ok(P, k_in, k, n);
+    if (rc != TOPK_EF_OK) return rc;
+    if (k_in > 0 && (!in_idx || !in_val || bad_fp32_ptr(in_idx) || bad_fp32_ptr(in_val)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (k > 0 && (!out_idx || !out_val || bad_fp32_ptr(out_idx) || bad_fp32_ptr(out_val)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (!out_count || !ws || ((uintptr_t)ws % ALIGN) != 0 || bad_fp32_ptr(out_count))
+        return TOPK_EF_ERR_INVALID_ARG;
+    const MLayout L = merge_layout(P, k_in, k);
+    if (ws_bytes < L.total) return TOPK_EF_ERR_WORKSPACE;
+    DevFacts f;
+    if ((rc = device_facts(&f)) != TOPK_EF_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* w = (char*)ws;
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(w + L.ctrl);
+    uint32_t* sizes = reinterpret_cast<uint32_t*>(w + L.sizes);
+    uint32_t* bad = reinterpret_cast<uint32_t*>(w + L.bad);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
+    uint32_t* live = reinterpret_cast<uint32_t*>(w + L.live);
+    uint32_t* set_idx = reinterpret_cast<uint32_t*>(w + L.set_idx);
+    float* set_val = reinterpret_cast<float*>(w + L.set_val);
+    uint32_t* m_idx = reinterpret_cast<uint32_t*>(w + L.m_idx);
+    float* m_val = reinterpret_cast<float*>(w + L.m_val);
+    const bool single = (P == 1 || k_in == 0);
+    const uint32_t kernels = single ? 2u : (uint32_t)(1 + 2 * L.rounds);
+
+    MergeSetupParams sp;
+    memset(&sp, 0, sizeof(sp));
+    sp.in_idx = in_idx;
+    sp.in_val = in_val;
+    sp.P = P;
+    sp.k_in = k_in;
+    sp.n = n;
+    sp.ctrl = ctrl;
+    sp.kernels = kernels;
+    sp.zero_ptr = reinterpret_cast<uint4*>(w + L.zero_begin);
+    sp.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
+    sp.bad_words = bad;
+    sp.sizes = sizes;
+    sp.set_idx = set_idx;
+    sp.set_val = set_val;
+    sp.set_cap = L.cap;
+    sp.lonely = (!single && (P % 2 == 1)) ? P - 1 : -1;
+    sp.validate_blocks = L.vblocks;
+    const int nz = (int)std::max<uint64_t>(
+        1, std::min<uint64_t>(148, (sp.zero_vec4 + MZ_THREADS * 8 - 1) / (MZ_THREADS * 8)));
+    trace_before(st, "merge_setup_kernel");
+    merge_setup_kernel<<<L.vblocks + nz, MZ_THREADS, 0, st>>>(sp);
+    trace_after(st);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+
+    const int G = std::min(SLOT_MAX, f.sms * f.selm_blocks);
+    SelCommon cm;
+    cm.ctrl = ctrl;
+    cm.slots = reinterpret_cast<Slot*>(w + L.slots);
+
+    MergeSrc ms;
+    memset(&ms, 0, sizeof(ms));
+    ms.kmax = (uint32_t)std::min<int64_t>(k, 0xFFFFFFFFLL);
+    ms.out_idx = out_idx;
+    ms.out_val = out_val;
+    ms.out_count = out_count;
+    ms.out_k = k;
+    ms.set_idx = set_idx;
+    ms.set_val = set_val;
+    ms.set_cap = L.cap;
+    ms.sizes = sizes;
+    ms.bad_words = bad;
+    ms.n_bad = (int32_t)L.vblocks;
+
+    if (single) {
+        ms.m_idx = reinterpret_cast<const uint32_t*>(in_idx);
+        ms.m_val = in_val;
+        ms.mcap = k_in;
+        ms.T = 1;
+        ms.live = nullptr;
+        ms.live_const = (uint32_t)k_in;
+        ms.hist = hist;
+        ms.d1_done = 0;
+        ms.final_out = 1;
+        ms.pair_stride = 1;
+        cm.bar = &ctrl->merge_bar[0];
+        void* args[] = {&ms, &cm};
+        trace_before(st, "select_kernel<MergeSrc>");
+        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(G),
+                                        dim3(SEL_THREADS), args, 0, st);
+        trace_after(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        return TOPK_EF_OK;
+    }
+
+    for (int r = 0; r < L.rounds; ++r) {
+        MergeRoundParams mp;
+        mp.src_idx = r == 0 ? reinterpret_cast<const uint32_t*>(in_idx) : set_idx;
+        mp.src_val = r == 0 ? in_val : set_val;
+        mp.src_stride = r == 0 ? k_in : L.cap;
+        mp.sizes = r == 0 ? nullptr : sizes;
+        mp.size_const = (uint32_t)k_in;
+        mp.np = L.np[r];
+        mp.step = 1 << r;
+        mp.mcap = L.mcap[r];
+        mp.m_idx = m_idx;
+        mp.m_val = m_val;
+        mp.hist = hist + (size_t)L.pbase[r] * HIST_WORDS;
+        mp.live = live + L.pbase[r];
+        dim3 grid((unsigned)ceil_div64(L.mcap[r], MG_D), (unsigned)L.np[r]);
+        trace_before(st, "merge_round_kernel");
+        merge_round_kernel<<<grid, MG_THREADS, 0, st>>>(mp);
+        trace_after(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+
+        ms.m_idx = m_idx;
+        ms.m_val = m_val;
+        ms.mcap = L.mcap[r];
+        ms.T = L.np[r];
+        ms.live = mp.live;
+        ms.hist = mp.hist;
+        ms.d1_done = 1;
+        ms.final_out = (r == L.rounds - 1) ? 1 : 0;
+        ms.pair_stride = 2 << r;
+        if (r > 0) {
+            ms.bad_words = nullptr;
+            ms.n_bad = 0;
+        }
+        cm.bar = &ctrl->merge_bar[r];
+        void* args[] = {&ms, &cm};
+        trace_before(st, "select_kernel<MergeSrc>");
+        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(G),
+                                        dim3(SEL_THREADS), args, 0, st);
+        trace_after(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return TOPK_EF_OK;
+}
+
+int topk_ef_last_device_status(const void* ws, void* stream) {
+    if (!ws) return TOPK_EF_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t s = 0;
+    cudaError_t e = cudaMemcpyAsync(&s, ws, sizeof(s), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (s & ST_TIMEOUT) return TOPK_EF_ERR_DEVICE_TIMEOUT;
+    if (s & ST_BAD_INPUT) return TOPK_EF_ERR_BAD_INPUT;
+    if (s & ST_INCONSISTENT) return TOPK_EF_ERR_INTERNAL;
+    return TOPK_EF_OK;
+}
+
+int topk_ef_path_info(const void* ws, void* stream, int64_t* info) {
+    if (!ws || !info) return TOPK_EF_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Ctrl c;
+    cudaError_t e = cudaMemcpyAsync(&c, ws, sizeof(c), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    info[0] = c.mode;
+    info[1] = (int64_t)c.cand_total;
+    info[2] = (int64_t)c.cap;
+    info[3] = c.kernels;
+    return TOPK_EF_OK;
+}
+
+int topk_ef_last_cuda_error(void) { return t_last_cuda_error; }
+
+const char* topk_ef_status_string(int status) {
+    switch (status) {
+        case TOPK_EF_OK: return "ok";
+        case TOPK_EF_ERR_INVALID_ARG: return "invalid argument";
+        case TOPK_EF_ERR_WORKSPACE: return "workspace too small";
+        case TOPK_EF_ERR_CUDA: return "CUDA error";
+        case TOPK_EF_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case TOPK_EF_ERR_BAD_INPUT: return "malformed merge input";
+        case TOPK_EF_ERR_INTERNAL: return "internal count mismatch";
+        default: return "unknown status";
+    }
+}
+
+int topk_ef_set_test_flags(int flags) { return g_test_flags.exchange(flags); }
+
+int topk_ef_trace_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    int dev = 0;
+    cudaError_t e;
+    if (on) {
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e);
+        if (g_trace.dev != dev) {
+            if (g_trace.dev >= 0) {
+                int cur = dev;
+                cudaSetDevice(g_trace.dev);
+                for (auto& ev : g_trace.ev) cudaEventDestroy(ev);
+                cudaSetDevice(cur);
+            }
+            for (auto& ev : g_trace.ev)
+                if ((e = cudaEventCreate(&ev)) != cudaSuccess) return cuda_fail(e);
+            g_trace.dev = dev;
+        }
+    }
+    g_trace.on = on ? 1 : 0;
+    g_trace.n = 0;
+    return TOPK_EF_OK;
+}
+
+int topk_ef_trace_read(float* ms, const char** names, int max_entries, int* count) {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (!count || (max_entries > 0 && (!ms || !names))) return TOPK_EF_ERR_INVALID_ARG;
+    const int n = std::min(g_trace.n, std::max(0, max_entries));
+    *count = n;
+    for (int i = 0; i < n; ++i) {
+        cudaError_t e = cudaEventSynchronize(g_trace.ev[2 * i + 1]);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms[i], g_trace.ev[2 * i], g_trace.ev[2 * i + 1]);
+        if (e != cudaSuccess) return cuda_fail(e);
+        names[i] = g_trace.name[i];
+    }
+    g_trace.n = 0;
+    return TOPK_EF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,204 @@
+/*
+ * topk_ef.h -- C ABI of the B200 Top-k + error-feedback sparsifier and the
+ * gTop-k merge of sparse (index, value) sets.
+ *
+ * What the calls compute (sources are web pages, cited by title and section):
+ *
+ *  - One error-feedback step ("Sparsified SGD with Memory", abstract: send the
+ *    top-k entries and keep the accumulated error in memory; "The Convergence
+ *    of Sparsified Gradient Methods", abstract: transmit a subset by
+ *    magnitude, accumulate the rest locally):
+ *        acc[i]      = fmaf(lr, grad[i], residual[i])      (one fp32 rounding)
+ *        S           = the k indices of largest |acc|, ties to the lower index
+ *        out         = (i, acc[i]) for i in S, ascending i
+ *        residual[i] = +0.0f for i in S, acc[i] otherwise
+ *    |x| order is the order of bits(x) & 0x7FFFFFFF as an unsigned integer
+ *    (-0 == +0; NaN above +Inf).
+ *
+ *  - The gTop-k merge ("A Distributed Synchronous SGD Algorithm with Global
+ *    Top-k Sparsification for Low Bandwidth Networks", ABSTRACT: the global
+ *    top-k largest absolute values from P workers; method section: a
+ *    tournament in O(log P) rounds).  Round r = 0, 1, ... while 2^r < P: every
+ *    worker i that is a multiple of 2^(r+1) with i + 2^r < P replaces its set
+ *    by the top min(k, |U|) of U = S_i (+) S_{i+2^r}, the union with one fp32
+ *    add (round to nearest even) at common indices.  A worker without a
+ *    partner in a round keeps its set.  The result is the top min(k, |S_0|)
+ *    of S_0, ascending index.
+ *
+ * Conventions shared by every call:
+ *  - Pointers marked "device" are CUDA device pointers on the current device;
+ *    pointers marked "host" are host memory read before the call returns.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    compute call is asynchronous on that stream and returns once its work
+ *    is enqueued.
+ *  - The caller owns every buffer, including the workspace `ws`
+ *    (device memory, at least the size the matching *_workspace_bytes call
+ *    returns, 256-byte aligned).  Calls on the same workspace must be ordered
+ *    (same stream, or synchronised); the library allocates no memory and
+ *    keeps nothing between calls except inside `ws`.
+ *  - fp32 arrays must be 4-byte aligned; 16-byte aligned grad/residual take
+ *    the vectorised path, other alignments a scalar path with identical
+ *    results.
+ *  - Results are deterministic and bit-identical from run to run.
+ *
+ * Return codes.  The return value covers argument checks and launch errors;
+ * problems found on the device (a bounded wait that gave up, malformed merge
+ * input) are recorded in the workspace and read back with
+ * topk_ef_last_device_status().  No call traps, asserts on the device or
+ * waits without bound.
+ */
+#ifndef TOPK_EF_H
+#define TOPK_EF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TOPK_EF_OK 0
+/* null pointer, n < 0, k < 0, k > n, n > 2^31 - 1, T < 1, P < 1, k_in > n,
+   offsets not starting at 0 or decreasing, misaligned fp32 pointer */
+#define TOPK_EF_ERR_INVALID_ARG (-1)
+/* ws_bytes smaller than the matching *_workspace_bytes() */
+#define TOPK_EF_ERR_WORKSPACE (-2)
+/* a CUDA launch or runtime call failed; topk_ef_last_cuda_error() has it */
+#define TOPK_EF_ERR_CUDA (-3)
+/* device: a bounded spin-wait gave up (outputs are undefined) */
+#define TOPK_EF_ERR_DEVICE_TIMEOUT (-4)
+/* device: merge input rows not strictly ascending or indices outside [0, n) */
+#define TOPK_EF_ERR_BAD_INPUT (-5)
+/* device: an internal count did not add up (outputs are undefined) */
+#define TOPK_EF_ERR_INTERNAL (-6)
+
+/* ---------------------------------------------------------------- compress */
+
+/* Workspace bytes for topk_ef_compress on n elements with k kept.
+   Returns 0 for invalid (n, k). */
+size_t topk_ef_workspace_bytes(int64_t n, int64_t k);
+
+/*
+ * One error-feedback step on a flat fp32 tensor.
+ *   grad      device, fp32[n], read only; must not overlap residual or outputs
+ *   residual  device, fp32[n]; in: the memory, out: acc with the k sent slots
+ *             set to +0.0f
+ *   n         0 <= n <= 2^31 - 1 (indices are int32)
+ *   lr        scale applied to grad inside the single fmaf
+ *   k         0 <= k <= n
+ *   out_idx   device, int32[k], ascending indices of the sent entries
+ *   out_val   device, fp32[k], acc at those indices (signed)
+ *   ws        device workspace of ws_bytes >= topk_ef_workspace_bytes(n, k)
+ */
+int topk_ef_compress(const float* grad, float* residual, int64_t n, float lr,
+                     int64_t k, int32_t* out_idx, float* out_val, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Workspace bytes for topk_ef_compress_batched with the same (offsets, k, T).
+   offsets and k are host arrays.  Returns 0 for invalid arguments. */
+size_t topk_ef_batched_workspace_bytes(const int64_t* offsets,
+                                       const int64_t* k, int32_t T);
+
+/*
+ * One error-feedback step on each of T tensors stored back to back in one
+ * flat bucket (per-tensor k; the tensors are independent problems).
+ *   grad, residual  device, fp32[offsets[T]]; tensor l is
+ *                   [offsets[l], offsets[l+1]); residual updated in place
+ *   offsets         host, int64[T+1], offsets[0] = 0, non-decreasing,
+ *                   offsets[T] <= 2^31 - 1
+ *   k               host, int64[T], 0 <= k[l] <= offsets[l+1] - offsets[l]
+ *   T               number of tensors, >= 1
+ *   out_idx         device, int32[sum k]; tensor l's entries start at
+ *                   sum_{j<l} k[j] and hold indices LOCAL to tensor l,
+ *                   ascending
+ *   out_val         device, fp32[sum k], matching acc values
+ *   ws              device workspace of ws_bytes >=
+ *                   topk_ef_batched_workspace_bytes(offsets, k, T)
+ */
+int topk_ef_compress_batched(const float* grad, float* residual,
+                             const int64_t* offsets, const int64_t* k,
+                             int32_t T, float lr, int32_t* out_idx,
+                             float* out_val, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* ------------------------------------------------------------------ merge */
+
+/* Workspace bytes for gtopk_merge with P sets of k_in entries keeping k.
+   Returns 0 for invalid arguments. */
+size_t gtopk_merge_workspace_bytes(int32_t P, int64_t k_in, int64_t k);
+
+/*
+ * gTop-k tournament over P sparse sets (P workers simulated on one GPU).
+ *   in_idx     device, int32[P][k_in], each row strictly ascending, values in
+ *              [0, n) (checked on the device: TOPK_EF_ERR_BAD_INPUT)
+ *   in_val     device, fp32[P][k_in]
+ *   P          number of workers, 1 <= P <= 512
+ *   k_in       entries per input set, 0 <= k_in <= n
+ *   k          entries kept per round and in the result, k >= 0
+ *   n          index bound
+ *   out_idx    device, int32[k]; the result in ascending index order; slots
+ *              past the result length hold -1
+ *   out_val    device, fp32[k]; the summed values; slots past the length 0
+ *   out_count  device, int32[1]; the result length min(k, |S_0|)
+ *   ws         device workspace of ws_bytes >=
+ *              gtopk_merge_workspace_bytes(P, k_in, k)
+ */
+int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P,
+                int64_t k_in, int64_t k, int64_t n, int32_t* out_idx,
+                float* out_val, int32_t* out_count, void* ws, size_t ws_bytes,
+                void* stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronises `stream` and returns the device-side status of the last call
+   that used `ws`: TOPK_EF_OK, TOPK_EF_ERR_DEVICE_TIMEOUT,
+   TOPK_EF_ERR_BAD_INPUT or TOPK_EF_ERR_INTERNAL (or TOPK_EF_ERR_CUDA if the
+   read-back failed). */
+int topk_ef_last_device_status(const void* ws, void* stream);
+
+/* The cudaError_t of the last TOPK_EF_ERR_CUDA returned on this thread. */
+int topk_ef_last_cuda_error(void);
+
+/* Human-readable name of a return code (static string). */
+const char* topk_ef_status_string(int status);
+
+/*
+ * Diagnostics of the last compress call on `ws` (synchronises `stream`):
+ *   info[0]  path taken: 0 = candidate prefilter, 1 = full rescan fallback
+ *   info[1]  candidates kept by the prefilter
+ *   info[2]  candidate capacity of the workspace
+ *   info[3]  kernels launched by that call
+ * `info` is host memory of 4 int64.  Returns a status code.
+ */
+int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
+
+/*
+ * Test hook, process wide: bit 0 forces the full rescan fallback of the
+ * compress calls; bit 1 forces the prefilter threshold of every tensor to 0
+ * (every element a candidate, which overflows the candidate capacity for
+ * large tensors and so also ends in the fallback).  0 restores normal
+ * behaviour.  Returns the previous flags.
+ */
+int topk_ef_set_test_flags(int flags);
+
+/*
+ * Tracing, process wide, for one thread at a time: while enabled, every
+ * kernel a compute call launches is bracketed by two CUDA events recorded on
+ * the call's stream (the library owns the events, created on the device that
+ * is current when tracing is enabled).  Up to 4096 launches are recorded;
+ * later ones are not.
+ *   topk_ef_trace_enable(1|0)   switch on / off (either clears the record)
+ *   topk_ef_trace_read(ms, names, max, &count)
+ *       waits for the recorded launches, writes the duration in milliseconds
+ *       (host float[max]) and kernel name (host const char*[max], static
+ *       strings) of the first min(max, recorded) of them, sets *count to that
+ *       number and clears the record.
+ */
+int topk_ef_trace_enable(int on);
+int topk_ef_trace_read(float* ms, const char** names, int max_entries, int* count);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOPK_EF_H */

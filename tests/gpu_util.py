@@ -1,0 +1,96 @@
+"""Helpers for the GPU parity tests: run the library and the oracle on the
+same seeded inputs and compare bit for bit."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import error_feedback_b200 as ef
+import oracle
+
+
+def bits(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def to_dev(a: np.ndarray, offset_elems: int = 0) -> torch.Tensor:
+    """Copy to cuda:0; with offset_elems > 0 the tensor is a view that starts
+    offset_elems elements into a larger buffer (to test misaligned bases)."""
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if offset_elems:
+        buf = torch.empty(a.size + offset_elems, dtype=t.dtype, device="cuda")
+        v = buf[offset_elems:]
+        v.copy_(t)
+        return v
+    return t.to("cuda")
+
+
+def assert_same_step(step, gi, gv, gres, oi, ov, ores):
+    gi = gi.cpu().numpy()
+    gv = gv.cpu().numpy()
+    gres = gres.cpu().numpy()
+    assert gi.shape == oi.shape, (step, gi.shape, oi.shape)
+    if not np.array_equal(gi, oi):
+        bad = np.nonzero(gi != oi)[0]
+        raise AssertionError(f"step {step}: {bad.size} index mismatches, first at {bad[0]}: "
+                             f"gpu {gi[bad[0]]} oracle {oi[bad[0]]}")
+    if not np.array_equal(bits(gv), bits(ov)):
+        bad = np.nonzero(bits(gv) != bits(ov))[0]
+        raise AssertionError(f"step {step}: {bad.size} value mismatches, first at {bad[0]}")
+    if not np.array_equal(bits(gres), bits(ores)):
+        bad = np.nonzero(bits(gres) != bits(ores))[0]
+        raise AssertionError(f"step {step}: {bad.size} residual mismatches, first at {bad[0]}: "
+                             f"gpu {gres[bad[0]]!r} oracle {ores[bad[0]]!r}")
+
+
+def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=None):
+    """EF steps on the GPU and in the oracle; every step compared.
+    grads: list of float32 arrays (one per step).  Returns the GPU residual."""
+    o = oracle.get()
+    n = grads[0].size
+    ores = np.zeros(n, np.float32) if res0 is None else res0.copy()
+    dres = to_dev(ores, offset_elems)
+    for s, g in enumerate(grads):
+        dg = to_dev(g, offset_elems)
+        gi, gv = ef.topk_ef_compress(dg, dres, lr, k, ws=ws)
+        st = ef.topk_ef_last_device_status(ws) if ws is not None else 0
+        assert st == 0, ef.status_string(st)
+        oi, ov = o.compress(g, ores, lr, k, backend)
+        assert_same_step(s, gi, gv, dres, oi, ov, ores)
+    return dres
+
+
+def run_batched_steps(grads, offsets, ks, lr, res0=None, backend=0, ws=None):
+    o = oracle.get()
+    N = int(offsets[-1])
+    ores = np.zeros(N, np.float32) if res0 is None else res0.copy()
+    dres = to_dev(ores)
+    for s, g in enumerate(grads):
+        dg = to_dev(g)
+        gi, gv = ef.topk_ef_compress_batched(dg, dres, offsets, ks, lr, ws=ws)
+        if ws is not None:
+            st = ef.topk_ef_last_device_status(ws)
+            assert st == 0, ef.status_string(st)
+        oi, ov = o.compress_batched(g, ores, offsets, ks, lr, backend)
+        assert_same_step(s, gi, gv, dres, oi, ov, ores)
+    return dres
+
+
+def run_merge(idx, val, k, n, ws=None):
+    o = oracle.get()
+    di = to_dev(idx)
+    dv = to_dev(val)
+    gi, gv, gc = ef.gtopk_merge(di, dv, k, n, ws=ws)
+    if ws is not None:
+        st = ef.topk_ef_last_device_status(ws)
+        assert st == 0, ef.status_string(st)
+    oi, ov = o.gtopk_merge(idx, val, k, n)
+    cnt = int(gc.cpu().item())
+    assert cnt == oi.size, (cnt, oi.size)
+    gi = gi.cpu().numpy()
+    gv = gv.cpu().numpy()
+    assert np.array_equal(gi[:cnt], oi), "merge index mismatch"
+    assert np.array_equal(bits(gv[:cnt]), bits(ov)), "merge value mismatch"
+    assert np.all(gi[cnt:] == -1) and np.all(bits(gv[cnt:]) == 0)
+    return gi, gv, cnt

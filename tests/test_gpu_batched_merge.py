@@ -1,0 +1,133 @@
+"""GPU parity of topk_ef_compress_batched and gtopk_merge against the oracle."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import error_feedback_b200 as ef
+from gpu_util import run_batched_steps, run_merge, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LR = np.float32(0.1)
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bucket(sizes, seed, scales=None):
+    rng = np.random.default_rng(seed)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    g = np.empty(int(offsets[-1]), np.float32)
+    for l, nl in enumerate(sizes):
+        s = scales[l] if scales is not None else 10.0 ** rng.uniform(-4, -1)
+        g[offsets[l]:offsets[l + 1]] = rng.laplace(0, s, nl).astype(np.float32)
+    return g, offsets
+
+
+def _wsb(offsets, ks):
+    return torch.empty(ef.topk_ef_batched_workspace_bytes(offsets, ks), dtype=torch.uint8,
+                       device="cuda")
+
+
+def test_batched_small_mixed():
+    sizes = [1, 0, 7, 8192, 8193, 100_000, 3, 70_001, 0, 5]
+    ks = [1, 0, 0, 8192, 9, 100, 3, 71, 0, 2]
+    grads = []
+    for s in range(3):
+        g, offsets = _bucket(sizes, 100 + s)
+        grads.append(g)
+    run_batched_steps(grads, offsets, ks, LR, ws=_wsb(offsets, ks))
+
+
+def test_batched_vgg16_scaled_down():
+    """VGG-16 layer structure with every tensor 1/64 of its size."""
+    sizes = [max(1, n // 64) for n in datagen.VGG16_SIZES]
+    ks = [(n + 999) // 1000 for n in sizes]
+    b = datagen.vgg16_scales()
+    grads = [_bucket(sizes, 200 + s, b)[0] for s in range(3)]
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    run_batched_steps(grads, offsets, ks, LR, ws=_wsb(offsets, ks))
+
+
+def test_batched_many_tensors():
+    """More tensors than one launch group holds (600 > 256)."""
+    rng = np.random.default_rng(9)
+    sizes = rng.integers(0, 3000, 600).tolist()
+    sizes[17] = 200_000
+    ks = [int(rng.integers(0, n + 1)) if n else 0 for n in sizes]
+    grads = [_bucket(sizes, 300 + s)[0] for s in range(2)]
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    run_batched_steps(grads, offsets, ks, LR, ws=_wsb(offsets, ks))
+
+
+def test_batched_vgg16_full():
+    """The full VGG-16 bucket (16 tensors, 138,344,128 elements), per-tensor
+    k = ceil(n_l / 1000); the first 2 of the 5 EF steps."""
+    grads = []
+    for s in range(2):
+        g, offsets, ks = datagen.vgg16_bucket(s)
+        grads.append(g)
+    ws = _wsb(offsets, ks)
+    run_batched_steps(grads, offsets, ks, LR, backend=1, ws=ws)
+    assert ef.topk_ef_path_info(ws)["fallback"] == 0
+
+
+# --------------------------------------------------------------------- merge
+
+def _mws(P, k_in, k):
+    return torch.empty(ef.gtopk_merge_workspace_bytes(P, k_in, k), dtype=torch.uint8,
+                       device="cuda")
+
+
+def test_merge_golden():
+    with open(os.path.join(GOLDEN, "merge_small.json")) as f:
+        g = json.load(f)
+    idx = np.array(g["idx"], np.int32)
+    val = np.array(g["val"], np.float32)
+    gi, gv, cnt = run_merge(idx, val, g["k"], g["n"], ws=_mws(4, 3, g["k"]))
+    assert gi[:cnt].tolist() == g["out_idx"] and gv[:cnt].tolist() == g["out_val"]
+
+
+@pytest.mark.parametrize("P,k_in,k,n", [
+    (1, 100, 50, 1000), (1, 100, 200, 1000), (2, 1000, 1000, 5000), (3, 500, 700, 3000),
+    (5, 800, 300, 4000), (8, 2000, 2000, 100_000), (13, 1000, 4000, 20_000),
+    (32, 3000, 3000, 1_000_000), (4, 0, 10, 100), (6, 10, 0, 100), (7, 5000, 100, 6000),
+    (2, 5000, 10_000, 10_000),
+])
+def test_merge_shapes(P, k_in, k, n):
+    idx, val = datagen.gtopk_sets(P=P, k=k_in, n=n, step=P + k) if k_in else (
+        np.zeros((P, 0), np.int32), np.zeros((P, 0), np.float32))
+    run_merge(idx, val, k, n, ws=_mws(P, k_in, k))
+
+
+def test_merge_heavy_overlap():
+    """Every set drawn from one small pool: most indices collide."""
+    rng = np.random.default_rng(21)
+    P, k_in, n = 16, 900, 1000
+    idx = np.stack([np.sort(rng.choice(n, k_in, replace=False)) for _ in range(P)]).astype(np.int32)
+    val = rng.choice(np.array([0.5, -0.5, 1.0, 0.25], np.float32), (P, k_in))
+    run_merge(idx, val, 400, n, ws=_mws(P, k_in, 400))
+
+
+def test_merge_resnet50_32_workers():
+    """P = 32 workers, k = 25,557 of n = 25,557,032 each, half from a shared
+    hot set of 2k indices; 5 rounds."""
+    idx, val = datagen.gtopk_sets()
+    ws = _mws(32, idx.shape[1], 25_557)
+    run_merge(idx, val, 25_557, datagen.RESNET50_N, ws=ws)
+
+
+def test_merge_bad_input_flagged():
+    idx = np.array([[1, 5, 3], [0, 2, 4]], np.int32)   # row 0 not ascending
+    val = np.ones((2, 3), np.float32)
+    ws = _mws(2, 3, 3)
+    ef.gtopk_merge(to_dev(idx), to_dev(val), 3, 10, ws=ws)
+    assert ef.topk_ef_last_device_status(ws) == ef.ERR_BAD_INPUT
+    idx2 = np.array([[1, 5, 30], [0, 2, 4]], np.int32)  # index >= n
+    ef.gtopk_merge(to_dev(idx2), to_dev(val), 3, 10, ws=ws)
+    assert ef.topk_ef_last_device_status(ws) == ef.ERR_BAD_INPUT
+    good = np.array([[1, 3, 5], [0, 2, 4]], np.int32)
+    ef.gtopk_merge(to_dev(good), to_dev(val), 3, 10, ws=ws)
+    assert ef.topk_ef_last_device_status(ws) == 0

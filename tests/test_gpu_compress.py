@@ -1,0 +1,149 @@
+"""GPU parity of topk_ef_compress against the CPU oracle (bit-exact: identical
+index sets, values and residuals at 0 ULP, every error-feedback step)."""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import error_feedback_b200 as ef
+from gpu_util import bits, run_compress_steps, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LR = np.float32(0.1)
+
+
+def _ws(n, k):
+    return torch.empty(ef.topk_ef_workspace_bytes(n, k), dtype=torch.uint8, device="cuda")
+
+
+def test_flat_normal_1m():
+    """1,048,576 elements, N(0,1), k = 1,048, three EF steps with fresh
+    gradients (the 1M flat workload)."""
+    n, k = 1 << 20, 1048
+    grads = [datagen.flat_normal(s) for s in range(3)]
+    ws = _ws(n, k)
+    run_compress_steps(grads, LR, k, ws=ws)
+    assert ef.topk_ef_path_info(ws)["fallback"] == 0
+
+
+@pytest.mark.parametrize("n,k", [
+    (1, 1), (1, 0), (2, 1), (5, 5), (31, 7), (1000, 1), (1000, 999), (8191, 100),
+    (8192, 8192), (8193, 3), (65535, 65), (65537, 66), (100003, 100), (300001, 3000),
+    (2_000_003, 2), (777_777, 77_777),
+])
+def test_shapes(n, k):
+    rng = np.random.default_rng(n * 7 + k)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(2)]
+    res0 = (rng.standard_normal(n) * 0.05).astype(np.float32)
+    run_compress_steps(grads, LR, k, res0=res0, ws=_ws(n, k))
+
+
+def test_empty():
+    ws = _ws(0, 0)
+    g = torch.empty(0, dtype=torch.float32, device="cuda")
+    r = torch.empty(0, dtype=torch.float32, device="cuda")
+    i, v = ef.topk_ef_compress(g, r, LR, 0, ws=ws)
+    assert i.numel() == 0 and ef.topk_ef_last_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("n,k", [(200_001, 5000), (1_000_000, 123_457), (70_000, 1)])
+def test_heavy_ties(n, k):
+    """Magnitudes from a handful of values: the threshold is shared by
+    thousands of entries and the lower indices must win."""
+    rng = np.random.default_rng(n + k)
+    pool = np.array([0.5, -0.5, 1.0, -1.0, 0.25, 2.0, -2.0, 0.0], np.float32)
+    grads = [rng.choice(pool, n) for _ in range(3)]
+    run_compress_steps(grads, np.float32(1.0), k, ws=_ws(n, k))
+
+
+def test_all_equal_magnitude():
+    n, k = 150_000, 4321
+    rng = np.random.default_rng(3)
+    g = np.where(rng.random(n) < 0.5, np.float32(0.75), np.float32(-0.75)).astype(np.float32)
+    run_compress_steps([g], np.float32(1.0), k, ws=_ws(n, k))
+
+
+def test_special_values():
+    """NaN, +-Inf, +-0 and subnormals mixed into a normal gradient."""
+    n, k = 120_001, 1200
+    rng = np.random.default_rng(5)
+    g = rng.standard_normal(n).astype(np.float32)
+    sp = np.array([np.nan, np.inf, -np.inf, 0.0, -0.0, 1e-45, -1e-45, 1e-40, 3e38, -3e38],
+                  np.float32)
+    pos = rng.choice(n, 500, replace=False)
+    g[pos] = rng.choice(sp, 500)
+    res0 = np.zeros(n, np.float32)
+    res0[rng.choice(n, 100, replace=False)] = np.float32(-0.0)
+    run_compress_steps([g, g], np.float32(1.0), k, res0=res0, ws=_ws(n, k))
+
+
+@pytest.mark.parametrize("offset", [1, 2, 3])
+def test_unaligned_base(offset):
+    """grad/residual not 16-byte aligned: the scalar path must agree."""
+    n, k = 300_007, 301
+    rng = np.random.default_rng(offset)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(2)]
+    run_compress_steps(grads, LR, k, offset_elems=offset, ws=_ws(n, k))
+
+
+@pytest.mark.parametrize("flags", [1, 2])
+def test_forced_fallback(flags):
+    """bit 0: force the residual rescan; bit 1: prefilter threshold 0, which
+    overflows the candidate capacity and so also ends in the rescan."""
+    n, k = 3_000_017, 3000
+    rng = np.random.default_rng(11 + flags)
+    grads = [rng.laplace(0, 1e-3, n).astype(np.float32) for _ in range(2)]
+    ws = _ws(n, k)
+    old = ef.topk_ef_set_test_flags(flags)
+    try:
+        run_compress_steps(grads, LR, k, ws=ws)
+        info = ef.topk_ef_path_info(ws)
+    finally:
+        ef.topk_ef_set_test_flags(old)
+    assert info["fallback"] == 1, info
+
+
+def test_sampler_defeated():
+    """Only the strided sample positions hold large values, so the threshold
+    estimate sits above the k-th magnitude (fewer than k candidates): the
+    rescan fallback must give the exact answer."""
+    n, k = 4_000_000, 20_000
+    g = np.full(n, 1e-6, np.float32)
+    m = 16384
+    sampled = (np.arange(m, dtype=np.int64) * n) // m
+    mask = np.ones(n, bool)
+    mask[sampled] = False
+    pos = np.nonzero(mask)[0][::7][:50_000]
+    g[pos] = np.float32(1.0) + np.arange(pos.size, dtype=np.float32) * np.float32(1e-4)
+    g[sampled] = np.float32(10.0)
+    ws = _ws(n, k)
+    run_compress_steps([g], np.float32(1.0), k, ws=ws)
+    info = ef.topk_ef_path_info(ws)
+    assert info["fallback"] == 1 and info["candidates"] < k, info
+
+
+def test_deterministic():
+    n, k = 5_000_000, 5000
+    g = datagen.laplace(n, 77, 1e-3)
+    out = []
+    for _ in range(2):
+        dg = to_dev(g)
+        dr = torch.zeros(n, dtype=torch.float32, device="cuda")
+        i, v = ef.topk_ef_compress(dg, dr, LR, k)
+        out.append((i.cpu().numpy(), bits(v.cpu().numpy()), bits(dr.cpu().numpy())))
+    for a, b in zip(out[0], out[1]):
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("density", [1e-2, 1e-3, 1e-4])
+def test_resnet50_mix_full(density):
+    """n = 25,557,032 (ResNet-50 sized) mixed Laplace / Student-t gradient,
+    k = floor(density * n); the first 3 of the 10 EF steps."""
+    n = datagen.RESNET50_N
+    k = datagen.density_k(n, density)
+    grads = [datagen.resnet50_mix(s) for s in range(3)]
+    ws = _ws(n, k)
+    run_compress_steps(grads, LR, k, backend=1, ws=ws)
+    info = ef.topk_ef_path_info(ws)
+    assert info["fallback"] == 0, info
