@@ -152,16 +152,25 @@ def gtopk_sets(P: int = 32, k: int = 25_557, n: int = RESNET50_N, config: int = 
     hot_mask[hot] = True
     idx = np.empty((P, k), dtype=np.int32)
     val = np.empty((P, k), dtype=np.float32)
+    if k > n:
+        raise ValueError("k > n")
     khot = min(k // 2, nhot)
     for p in range(P):
         r = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 1 + p])))
         a = r.choice(hot, size=khot, replace=False)
         need = k - khot
-        rest = np.empty(0, dtype=np.int64)
-        while rest.size < need:
-            cand = r.integers(0, n, size=2 * (need - rest.size) + 16)
-            cand = cand[~hot_mask[cand]]
-            rest = np.unique(np.concatenate([rest, cand]))
+        if n - nhot >= 4 * need:
+            # rejection sampling over the indices outside the hot set
+            rest = np.empty(0, dtype=np.int64)
+            while rest.size < need:
+                cand = r.integers(0, n, size=2 * (need - rest.size) + 16)
+                cand = cand[~hot_mask[cand]]
+                rest = np.unique(np.concatenate([rest, cand]))
+        else:
+            # small index space: draw from every index not taken yet
+            taken = np.zeros(n, dtype=bool)
+            taken[a] = True
+            rest = np.nonzero(~taken)[0]
         if rest.size > need:
             rest = r.choice(rest, size=need, replace=False)
         s = np.sort(np.concatenate([a.astype(np.int64), rest]))
