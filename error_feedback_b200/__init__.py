@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.topk_ef_status_string.restype = ctypes.c_char_p
         L.topk_ef_path_info.argtypes = [_vp, _vp, _pi64]
         L.topk_ef_path_info.restype = ctypes.c_int
+        L.topk_ef_phase_times.argtypes = [_vp, _vp, _pi64]
+        L.topk_ef_phase_times.restype = ctypes.c_int
         L.topk_ef_set_test_flags.argtypes = [ctypes.c_int]
         L.topk_ef_set_test_flags.restype = ctypes.c_int
         L.topk_ef_trace_enable.argtypes = [ctypes.c_int]
@@ -237,6 +239,13 @@ def topk_ef_path_info(ws, stream=None) -> dict:
     _check(lib().topk_ef_path_info(ws.data_ptr(), _stream(stream), info), "topk_ef_path_info")
     return {"fallback": int(info[0]), "candidates": int(info[1]), "capacity": int(info[2]),
             "kernels": int(info[3])}
+
+
+def topk_ef_phase_times(ws, stream=None) -> list:
+    """Select kernel phase end times (ns from its start; -1: phase not run)."""
+    ns = (ctypes.c_int64 * 8)()
+    _check(lib().topk_ef_phase_times(ws.data_ptr(), _stream(stream), ns), "topk_ef_phase_times")
+    return [int(x) for x in ns]
 
 
 def topk_ef_set_test_flags(flags: int) -> int:

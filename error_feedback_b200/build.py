@@ -4,6 +4,7 @@
 """
 from __future__ import annotations
 
+import glob
 import os
 import subprocess
 import sys
@@ -11,9 +12,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "topk_ef.cu")
-DEPS = [os.path.join(HERE, "csrc", f) for f in
-        ("common.cuh", "kernels_compress.cuh", "kernels_select.cuh", "kernels_merge.cuh",
-         "topk_ef.cu")] + [os.path.join(ROOT, "include", "topk_ef.h")]
+DEPS = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu*"))) + [
+    os.path.join(ROOT, "include", "topk_ef.h")]
 LIB = os.path.join(HERE, "libtopk_ef.so")
 
 NVCC_FLAGS = [

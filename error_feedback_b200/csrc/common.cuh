@@ -1,8 +1,8 @@
 // Device helpers shared by the Top-k + error-feedback kernels.
 //
-// |x| order: key(x) = bits(x) & 0x7FFFFFFF compared as an unsigned integer.
-// This equals the order of |x| for every non-NaN value (-0 == +0) and puts
-// NaN above +Inf, so "the k entries of largest absolute value" ("A
+// |x| order: key(x) = bits(x) & 0x7FFFFFFF compared as an unsigned integer,
+// with every NaN mapped to 0x7FFFFFFF.  This equals the order of |x| for every
+// non-NaN value (-0 == +0) and puts all NaNs, as one value, above +Inf, so "the k entries of largest absolute value" ("A
 // Distributed Synchronous SGD Algorithm with Global Top-k Sparsification for
 // Low Bandwidth Networks", ABSTRACT) is a total order once ties go to the
 // lower index.
@@ -44,11 +44,21 @@ struct Ctrl {
     uint32_t pad0;
     uint32_t merge_bar[32]; // grid barrier counters, one per merge round
     uint32_t pad1[6];
+    uint64_t t_phase[8];    // select kernel: globaltimer at each phase (block 0)
 };
-static_assert(sizeof(Ctrl) == 192, "Ctrl layout");
+static_assert(sizeof(Ctrl) == 256, "Ctrl layout");
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Every NaN gets the largest key (NaN payloads are implementation-defined:
+// an fma on the GPU returns the canonical NaN, other sources may not).
 __device__ __forceinline__ uint32_t key_of(float x) {
-    return __float_as_uint(x) & KEY_MASK;
+    const uint32_t k = __float_as_uint(x) & KEY_MASK;
+    return k > 0x7F800000u ? KEY_MASK : k;
 }
 
 __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {

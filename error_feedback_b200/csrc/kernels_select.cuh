@@ -53,13 +53,18 @@ struct CompressSrc {
     int64_t N;
     int32_t T;
     const SegMeta* meta;
-    const int64_t* cand_start;   // [T+1]
-    const uint32_t* cand_idx;
-    const float* cand_val;
+    int64_t* cand_start;         // [T+1], built by the gather phase
+    uint32_t* cand_idx;          // dense candidate list, index order
+    float* cand_val;
     uint64_t cap;
     uint32_t* hist;              // [T][HIST_WORDS]
     int32_t* out_idx;
     float* out_val;
+    uint32_t num_wt;             // warp tiles of the streaming pass
+    const uint32_t* wt_count;
+    const uint32_t* st_idx;      // [num_wt][WT_CAP]
+    const float* st_val;
+    const uint32_t* bound_before;
     int32_t force_dense;
     int32_t dense;               // decided inside the kernel
 
@@ -80,18 +85,6 @@ struct CompressSrc {
         out_val[m.out_base + rank] = val;
         resid[idx] = 0.0f;
     }
-    // Block-uniform decision: the prefilter holds the top-k of every tensor
-    // when each tensor kept at least k candidates and nothing was dropped.
-    __device__ void prepare(uint32_t* s_red, Ctrl* ctrl) {
-        const uint64_t total = (uint64_t)cand_start[T];
-        uint32_t bad = 0;
-        for (int l = threadIdx.x; l < T; l += blockDim.x)
-            bad |= (uint64_t)(cand_start[l + 1] - cand_start[l]) < (uint64_t)meta[l].k;
-        bad = block_sum(bad, s_red);
-        dense = (force_dense || total > cap || bad) ? 1 : 0;
-        if (blockIdx.x == 0 && threadIdx.x == 0) ctrl->mode = dense;
-    }
-    __device__ void finalize(const Resolved*) const {}
 };
 
 // Merge round: merged lists of the pairs (DEAD marks empty slots).
@@ -143,7 +136,7 @@ struct MergeSrc {
             set_val[s] = val;
         }
     }
-    __device__ void prepare(uint32_t*, Ctrl* ctrl) {
+    __device__ void fold_bad_input(Ctrl* ctrl) const {
         if (bad_words && blockIdx.x == 0 && threadIdx.x == 0) {
             uint32_t any = 0;
             for (int i = 0; i < n_bad; ++i) any |= bad_words[i];
@@ -249,13 +242,142 @@ __device__ __forceinline__ bool in_class(uint32_t key, int d, uint32_t prefix) {
     return d == 1 ? true : (d == 2 ? ((key >> 20) == prefix) : ((key >> 10) == prefix));
 }
 
+// Phase timestamps (block 0 only) for the diagnostics call.
+__device__ __forceinline__ void mark_phase(Ctrl* ctrl, int i) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) ctrl->t_phase[i] = global_ns();
+}
+
+// Gather phase of the compress select: rebuild the global candidate order
+// from the streaming pass's per-warp-tile staging.  Each block takes a
+// contiguous chunk of warp tiles; a grid barrier turns the chunk sums into
+// offsets; every staged candidate is copied to its place in the dense list,
+// and a warp tile that had more than WT_CAP candidates is rescanned from the
+// residual (which holds acc) with the same predicate.  Also records where each
+// tensor's candidates start.  Then decides the path for every block alike:
+// candidates only if each tensor kept at least k of them and the list fit.
+// Returns false if a barrier gave up.
+__device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
+                                int* s_flag, uint32_t* s_red, uint64_t* s_scan,
+                                int64_t* s_off, uint32_t* s_T0, uint32_t* s_scratch) {
+    const int G = gridDim.x, c = blockIdx.x, tid = threadIdx.x;
+    const uint32_t lane = lane_id(), warp = warp_id(), nwarps = blockDim.x >> 5;
+    const int T = src.T;
+    uint32_t* status = &cm.ctrl->status;
+    for (int l = tid; l < T; l += blockDim.x) {
+        s_off[l] = src.meta[l].off;
+        s_T0[l] = src.meta[l].T0;
+    }
+    if (tid == 0) s_off[T] = src.N;
+    const uint32_t W = src.num_wt;
+    const uint32_t per = (W + G - 1) / G;
+    const uint32_t w0 = min((uint32_t)c * per, W), w1 = min(w0 + per, W);
+    uint32_t mine = 0;
+    for (uint32_t w = w0 + tid; w < w1; w += blockDim.x) mine += src.wt_count[w];
+    mine = block_sum(mine, s_red);
+    if (tid == 0) cm.slots[c].gt_first = mine;
+    if (!grid_barrier(cm.bar, epoch, status, s_flag)) return false;
+    mark_phase(cm.ctrl, 1);
+
+    uint64_t before = 0, total = 0;
+    for (int i = tid; i < G; i += blockDim.x) {
+        const uint64_t v = cm.slots[i].gt_first;
+        total += v;
+        if (i < c) before += v;
+    }
+    before = block_sum(before, s_scan);
+    total = block_sum(total, s_scan);
+    const bool fits = total <= src.cap;
+    if (c == 0)
+        for (int l = tid; l <= T; l += blockDim.x)
+            if (l == 0) src.cand_start[0] = 0;
+            else if (s_off[l] >= src.N) src.cand_start[l] = (int64_t)total;
+
+    // overflow list in scratch: pairs (warp tile, offset)
+    uint32_t* s_ovf_w = s_scratch;
+    uint64_t* s_ovf_o = reinterpret_cast<uint64_t*>(s_scratch + SEL_THREADS);
+    uint32_t* s_ovf_n = s_scratch + 3 * SEL_THREADS;
+    uint64_t run = before;
+    for (uint32_t pw = w0; pw < w1; pw += blockDim.x) {
+        const uint32_t w = pw + tid;
+        const uint32_t cnt = w < w1 ? src.wt_count[w] : 0u;
+        if (tid == 0) *s_ovf_n = 0;
+        uint32_t piece;
+        const uint32_t ex = block_excl_scan(cnt, s_red, &piece);
+        const uint64_t off = run + ex;
+        if (w < w1) {
+            const int64_t base = (int64_t)w * WT;
+            const int64_t tend = min(base + (int64_t)WT, src.N);
+            if (T > 1)
+                for (int l = max(1, lower_bound_off(s_off, T, base)); l < T && s_off[l] < tend; ++l)
+                    src.cand_start[l] = (int64_t)(off + src.bound_before[l]);
+            if (fits && cnt) {
+                if (cnt <= WT_CAP) {
+                    for (uint32_t i = 0; i < cnt; ++i) {
+                        src.cand_idx[off + i] = src.st_idx[(size_t)w * WT_CAP + i];
+                        src.cand_val[off + i] = src.st_val[(size_t)w * WT_CAP + i];
+                    }
+                } else {
+                    const uint32_t slot = atomicAdd(s_ovf_n, 1u);
+                    s_ovf_w[slot] = w;
+                    s_ovf_o[slot] = off;
+                }
+            }
+        }
+        __syncthreads();
+        const uint32_t novf = *s_ovf_n;
+        for (uint32_t i = warp; i < novf; i += nwarps) {
+            const uint32_t w2 = s_ovf_w[i];
+            uint64_t pos = s_ovf_o[i];
+            const int64_t base = (int64_t)w2 * WT;
+            const int64_t tend = min(base + (int64_t)WT, src.N);
+            int l = seg_of(s_off, T, base);
+            for (int64_t e0 = base; e0 < tend; e0 += 32) {
+                const int64_t e = e0 + lane;
+                bool f = false;
+                float v = 0.f;
+                if (e < tend) {
+                    while (l < T - 1 && s_off[l + 1] <= e) ++l;
+                    v = src.resid[e];
+                    f = key_of(v) >= s_T0[l];
+                }
+                const uint32_t m = __ballot_sync(0xFFFFFFFFu, f);
+                if (f) {
+                    const uint64_t q = pos + __popc(m & ((1u << lane) - 1u));
+                    if (q < src.cap) {
+                        src.cand_idx[q] = (uint32_t)e;
+                        src.cand_val[q] = v;
+                    }
+                }
+                pos += __popc(m);
+                // keep the lanes' tensor cursors in step
+                l = __shfl_sync(0xFFFFFFFFu, l, 31);
+            }
+        }
+        __syncthreads();
+        run += piece;
+    }
+    if (!grid_barrier(cm.bar, epoch, status, s_flag)) return false;
+    mark_phase(cm.ctrl, 2);
+
+    uint32_t bad = 0;
+    for (int l = tid; l < T; l += blockDim.x)
+        bad |= (uint64_t)(src.cand_start[l + 1] - src.cand_start[l]) < (uint64_t)src.meta[l].k;
+    bad = block_sum(bad, s_red);
+    src.dense = (src.force_dense || !fits || bad) ? 1 : 0;
+    if (c == 0 && tid == 0) {
+        cm.ctrl->mode = src.dense;
+        cm.ctrl->cand_total = total;
+    }
+    return true;
+}
+
 // ---------------------------------------------------------------- kernel
 
 template <class Src>
 __global__ void __launch_bounds__(SEL_THREADS)
 select_kernel(Src src, SelCommon cm) {
     __shared__ int64_t s_seg[SEG_MAX + 1];
-    __shared__ uint32_t s_stage[D1_BINS + D2_BINS + D3_BINS];
+    __shared__ __align__(16) uint32_t s_stage[D1_BINS + D2_BINS + D3_BINS];
     __shared__ uint32_t s_h1[D1_BINS];
     __shared__ uint64_t s_scan[33];
     __shared__ uint32_t s_red[33];
@@ -268,8 +390,16 @@ select_kernel(Src src, SelCommon cm) {
     const int G = gridDim.x;
     uint32_t epoch = 0;
     uint32_t* status = &cm.ctrl->status;
+    mark_phase(cm.ctrl, 0);
 
-    src.prepare(s_red, cm.ctrl);
+    if constexpr (std::is_same<Src, CompressSrc>::value) {
+        __shared__ uint32_t s_T0[TCAP_LARGE];
+        if (!compress_gather(src, cm, epoch, &s_flag, s_red, s_scan, s_seg, s_T0, s_stage))
+            return;
+        __syncthreads();
+    } else {
+        src.fold_bad_input(cm.ctrl);
+    }
     const int T = src.nseg();
     for (int l = tid; l <= T; l += blockDim.x) s_seg[l] = src.seg_bound(l);
     __syncthreads();
@@ -318,6 +448,7 @@ select_kernel(Src src, SelCommon cm) {
             }
         }
         if (!grid_barrier(cm.bar, epoch, status, &s_flag)) return;
+        mark_phase(cm.ctrl, 2 + d);
     }
 
     // ---- per-block counts of (key > T, key == T) in the first and last segment
@@ -358,6 +489,7 @@ select_kernel(Src src, SelCommon cm) {
         if constexpr (std::is_same<Src, MergeSrc>::value) src.finalize_block0();
     }
     if (!grid_barrier(cm.bar, epoch, status, &s_flag)) return;
+    mark_phase(cm.ctrl, 6);
 
     // ---- emission
     for (int l = l_first; l <= l_last; ++l) {
@@ -442,6 +574,7 @@ select_kernel(Src src, SelCommon cm) {
             run_eq += (uint32_t)(tot & 0xFFFFFFFFu);
         }
     }
+    mark_phase(cm.ctrl, 7);
 }
 
 }  // namespace tke

@@ -154,10 +154,10 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
 
 // Workspace layout of one compress group (<= TCAP_LARGE tensors).
 struct CLayout {
-    size_t ctrl, meta, zero_begin, cand_start, hist, tile_status, zero_end, slots, cand_idx,
-        cand_val, total;
+    size_t ctrl, meta, zero_begin, cand_start, hist, zero_end, bound_before, wt_count, st_idx,
+        st_val, slots, cand_idx, cand_val, total;
     int64_t cap;
-    uint32_t num_tiles;
+    uint32_t num_wt;
 };
 
 CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
@@ -166,7 +166,7 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     int64_t cap = 0;
     for (const auto& p : plans) cap += p.cap;
     L.cap = cap;
-    L.num_tiles = (uint32_t)ceil_div64(N, TILE);
+    L.num_wt = (uint32_t)ceil_div64(N, WT);
     size_t o = 0;
     L.ctrl = o;
     o = align_up(o + sizeof(Ctrl));
@@ -177,9 +177,15 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + (T + 1) * sizeof(int64_t));
     L.hist = o;
     o = align_up(o + T * HIST_WORDS * sizeof(uint32_t));
-    L.tile_status = o;
-    o = align_up(o + (size_t)L.num_tiles * sizeof(uint64_t));
     L.zero_end = o;
+    L.bound_before = o;
+    o = align_up(o + (T + 1) * sizeof(uint32_t));
+    L.wt_count = o;
+    o = align_up(o + (size_t)L.num_wt * sizeof(uint32_t));
+    L.st_idx = o;
+    o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(uint32_t));
+    L.st_val = o;
+    o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(float));
     L.slots = o;
     o = align_up(o + SLOT_MAX * sizeof(Slot));
     L.cand_idx = o;
@@ -288,17 +294,18 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     sp.lr = lr;
     sp.T = T;
     sp.N = g.N;
-    sp.num_tiles = L.num_tiles;
+    sp.num_wt = L.num_wt;
     sp.meta = reinterpret_cast<const SegMeta*>(ws + L.meta);
     sp.ctrl = ctrl;
-    sp.tile_status = reinterpret_cast<uint64_t*>(ws + L.tile_status);
-    sp.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
-    sp.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
-    sp.cap = (uint64_t)L.cap;
+    sp.wt_count = reinterpret_cast<uint32_t*>(ws + L.wt_count);
+    sp.st_idx = reinterpret_cast<uint32_t*>(ws + L.st_idx);
+    sp.st_val = reinterpret_cast<float*>(ws + L.st_val);
     sp.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-    sp.cand_start = reinterpret_cast<int64_t*>(ws + L.cand_start);
+    sp.bound_before = reinterpret_cast<uint32_t*>(ws + L.bound_before);
     const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
-    const int g1 = (int)std::min<int64_t>(L.num_tiles, (int64_t)f.sms * f.k1_blocks);
+    const int64_t warps_needed = L.num_wt;
+    const int g1 = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(warps_needed, K1_THREADS / 32),
+                                                               (int64_t)f.sms * f.k1_blocks));
     trace_before(st, "stream_kernel");
     if (vec) stream_kernel<true><<<g1, K1_THREADS, 0, st>>>(sp);
     else stream_kernel<false><<<g1, K1_THREADS, 0, st>>>(sp);
@@ -311,13 +318,18 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     src.N = g.N;
     src.T = T;
     src.meta = sp.meta;
-    src.cand_start = sp.cand_start;
-    src.cand_idx = sp.cand_idx;
-    src.cand_val = sp.cand_val;
-    src.cap = sp.cap;
+    src.cand_start = reinterpret_cast<int64_t*>(ws + L.cand_start);
+    src.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
+    src.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
+    src.cap = (uint64_t)L.cap;
     src.hist = sp.hist;
     src.out_idx = out_idx;
     src.out_val = out_val;
+    src.num_wt = L.num_wt;
+    src.wt_count = sp.wt_count;
+    src.st_idx = sp.st_idx;
+    src.st_val = sp.st_val;
+    src.bound_before = sp.bound_before;
     src.force_dense = force_dense ? 1 : 0;
     src.dense = 0;
     SelCommon cm;
@@ -627,6 +639,18 @@ int topk_ef_path_info(const void* ws, void* stream, int64_t* info) {
     info[1] = (int64_t)c.cand_total;
     info[2] = (int64_t)c.cap;
     info[3] = c.kernels;
+    return TOPK_EF_OK;
+}
+
+int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns) {
+    if (!ws || !ns) return TOPK_EF_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Ctrl c;
+    cudaError_t e = cudaMemcpyAsync(&c, ws, sizeof(c), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (int i = 0; i < 8; ++i)
+        ns[i] = c.t_phase[i] ? (int64_t)(c.t_phase[i] - c.t_phase[0]) : -1;
     return TOPK_EF_OK;
 }
 

@@ -173,6 +173,15 @@ const char* topk_ef_status_string(int status);
 int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
 
 /*
+ * Diagnostics of the last call on `ws` (synchronises `stream`): for the
+ * select kernel's block 0, the time in nanoseconds from the kernel's start to
+ * the end of each phase: ns[1], ns[2] the two gather barriers (compress),
+ * ns[3..5] digit passes 1..3, ns[6] the count barrier, ns[7] the end of the
+ * emission; -1 for a phase that did not run.  `ns` is host memory of 8 int64.
+ */
+int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns);
+
+/*
  * Test hook, process wide: bit 0 forces the full rescan fallback of the
  * compress calls; bit 1 forces the prefilter threshold of every tensor to 0
  * (every element a candidate, which overflows the candidate capacity for

@@ -27,8 +27,9 @@
  *  - acc = fmaf(lr, grad, residual): lr times the gradient plus the memory,
  *    rounded once to fp32 (C99 fmaf is correctly rounded).
  *  - |x| order is the order of key(x) = bits(x) & 0x7FFFFFFF as an unsigned
- *    integer (equal to |x| order for all non-NaN values, -0 == +0, NaN above
- *    +Inf).
+ *    integer (equal to |x| order for all non-NaN values, -0 == +0); every NaN
+ *    has key 0x7FFFFFFF (above +Inf, all NaNs equal, whatever the payload:
+ *    NaN payloads and signs are implementation-defined in IEEE 754).
  *  - ties in |x| go to the lower index, so the selected set is unique.
  *  - output pairs (int32 index, fp32 signed value) in ascending index order.
  *  - the residual keeps acc at unselected slots and +0.0f at selected slots.
@@ -83,6 +84,8 @@ static uint32_t key_of(float x)
     uint32_t u = bits_of(x);
     return (u & 0x80000000u) ? (0x7FFFFFFFu - (u & 0x7FFFFFFFu)) / 2u : 0x3FFFFFFFu + (u >> 1);
 #else
+    /* every NaN orders as one value above +Inf, whatever its payload */
+    if (x != x) return 0x7FFFFFFFu;
     return bits_of(x) & 0x7FFFFFFFu;
 #endif
 }

@@ -193,6 +193,12 @@ def pin_special_cases(o, seed=14):
     x = np.array([1.0, np.inf, np.nan, -np.inf, 2.0], np.float32)
     assert o.select(x, 1).tolist() == [2]
     assert o.select(x, 3).tolist() == [1, 2, 3]
+    # every NaN is one value whatever its payload or sign: ties go to the
+    # lower index
+    nans = np.array([0x7FC00001, 0xFFC00000, 0x7FFFFFFF, 0xFF800001], np.uint32).view(np.float32)
+    x = np.array([5.0, nans[0], 7.0, nans[1], nans[2], nans[3]], np.float32)
+    assert o.select(x, 1).tolist() == [1]
+    assert o.select(x, 4).tolist() == [1, 3, 4, 5]
 
 
 def pin_backends_agree(o, seed=15):

@@ -147,3 +147,63 @@ def test_resnet50_mix_full(density):
     run_compress_steps(grads, LR, k, backend=1, ws=ws)
     info = ef.topk_ef_path_info(ws)
     assert info["fallback"] == 0, info
+
+
+@pytest.mark.slow
+def test_bf16_ties_1p5b_full():
+    """n = 1.5e9 (6 GB gradient + 6 GB residual), grad = bf16-rounded
+    N(0, 1e-3) so |acc| has heavy ties, k = 1,500,000, three EF steps; every
+    step compared bit for bit with the oracle (bounded-heap back-end).  The
+    oracle's residual is compared on the device to keep host memory down."""
+    import oracle
+    n, k = datagen.LARGE_N, 1_500_000
+    o = oracle.get()
+    ores = np.zeros(n, np.float32)
+    dres = torch.zeros(n, dtype=torch.float32, device="cuda")
+    ws = _ws(n, k)
+    for step in range(3):
+        g = datagen.bf16_normal(step)
+        dg = torch.from_numpy(g).cuda()
+        gi, gv = ef.topk_ef_compress(dg, dres, LR, k, ws=ws)
+        assert ef.topk_ef_last_device_status(ws) == 0
+        del dg
+        oi, ov = o.compress(g, ores, LR, k, 1)
+        del g
+        assert np.array_equal(gi.cpu().numpy(), oi), f"step {step}: index sets differ"
+        assert np.array_equal(bits(gv.cpu().numpy()), bits(ov)), f"step {step}: values differ"
+        dor = torch.from_numpy(ores).cuda()
+        same = torch.equal(dor.view(torch.int32), dres.view(torch.int32))
+        del dor
+        assert same, f"step {step}: residuals differ"
+    info = ef.topk_ef_path_info(ws)
+    assert info["fallback"] == 0, info
+
+
+@pytest.mark.parametrize("n,k", [(8192 * 3, 30), (1_000_003, 1000), (4_000_001, 4000),
+                                 (25_557_032, 25_557)])
+def test_tma_staged_stream(n, k):
+    """The TMA-staged streaming kernel (test flag bit 2) gives the same
+    results, including partial last tiles and lengths not divisible by 4."""
+    rng = np.random.default_rng(n % 1000 + 5)
+    grads = [rng.laplace(0, 1e-3, n).astype(np.float32) for _ in range(2)]
+    old = ef.topk_ef_set_test_flags(4)
+    try:
+        run_compress_steps(grads, LR, k, backend=1, ws=_ws(n, k))
+    finally:
+        ef.topk_ef_set_test_flags(old)
+
+
+def test_tma_staged_batched():
+    sizes = [1, 7, 70_001, 8192, 3, 250_000, 5]
+    ks = [1, 3, 70, 8192, 0, 250, 5]
+    rng = np.random.default_rng(44)
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    grads = [rng.laplace(0, 1e-2, int(offsets[-1])).astype(np.float32) for _ in range(2)]
+    from gpu_util import run_batched_steps
+    ws = torch.empty(ef.topk_ef_batched_workspace_bytes(offsets, ks), dtype=torch.uint8,
+                     device="cuda")
+    old = ef.topk_ef_set_test_flags(4)
+    try:
+        run_batched_steps(grads, offsets, ks, LR, ws=ws)
+    finally:
+        ef.topk_ef_set_test_flags(old)
