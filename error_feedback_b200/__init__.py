@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
         L.topk_ef_workspace_bytes.restype = _sz
         L.topk_ef_compress.argtypes = [_vp, _vp, _i64, ctypes.c_float, _i64, _vp, _vp, _vp, _sz, _vp]
         L.topk_ef_compress.restype = ctypes.c_int
+        L.topk_ef_compress_static.argtypes = [_vp, _vp, _i64, ctypes.c_float, _i64, _vp, _vp,
+                                              _vp]
+        L.topk_ef_compress_static.restype = ctypes.c_int
         L.topk_ef_batched_workspace_bytes.argtypes = [_pi64, _pi64, _i32]
         L.topk_ef_batched_workspace_bytes.restype = _sz
         L.topk_ef_compress_batched.argtypes = [_vp, _vp, _pi64, _pi64, _i32, ctypes.c_float, _vp, _vp,
@@ -156,6 +159,26 @@ def topk_ef_compress(grad, residual, lr, k, out_idx=None, out_val=None, ws=None,
                                 out_idx.data_ptr(), out_val.data_ptr(), ws.data_ptr(),
                                 ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "topk_ef_compress")
+    return out_idx, out_val
+
+
+def topk_ef_compress_static(grad, residual, lr, k, out_idx=None, out_val=None, stream=None):
+    """topk_ef_compress without a caller workspace: for callers that cannot
+    allocate device memory.  Uses the library's fixed 32 MiB scratch array
+    (shared by all calls; calls whose GPU work overlaps must not be issued)."""
+    _cuda_f32(grad, "grad")
+    _cuda_f32(residual, "residual")
+    if grad.numel() != residual.numel():
+        raise ValueError("grad and residual differ in size")
+    n, k = grad.numel(), int(k)
+    dev = grad.device
+    if out_idx is None:
+        out_idx = torch.empty(k, dtype=torch.int32, device=dev)
+    if out_val is None:
+        out_val = torch.empty(k, dtype=torch.float32, device=dev)
+    rc = lib().topk_ef_compress_static(grad.data_ptr(), residual.data_ptr(), n, float(lr), k,
+                                       out_idx.data_ptr(), out_val.data_ptr(), _stream(stream))
+    _check(rc, "topk_ef_compress_static")
     return out_idx, out_val
 
 

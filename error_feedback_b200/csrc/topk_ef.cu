@@ -348,6 +348,34 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
 
 bool bad_fp32_ptr(const void* p) { return ((uintptr_t)p & 3u) != 0; }
 
+// ------------------------------------------- compress without allocation
+// Scratch for topk_ef_compress_static: one array in the module's global
+// memory.  Each GPU that loads this library holds it until the process ends.
+// In host code `g_static_scratch` is only a host-side stand-in for the
+// symbol; the device address comes from cudaGetSymbolAddress, taken once per
+// device with that device current.
+constexpr size_t STATIC_SCRATCH_BYTES = TOPK_EF_STATIC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_static_scratch[STATIC_SCRATCH_BYTES];
+
+std::mutex g_static_mu;
+void* g_static_addr[64];
+
+int static_scratch_addr(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return TOPK_EF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_static_addr[dev] = ptr;
+    }
+    *out = g_static_addr[dev];
+    return TOPK_EF_OK;
+}
+
 // --------------------------------------------------------- merge planning
 
 struct MLayout {
@@ -469,6 +497,19 @@ int topk_ef_compress(const float* grad, float* residual, int64_t n, float lr, in
     const int64_t offsets[2] = {0, n};
     return topk_ef_compress_batched(grad, residual, offsets, &k, 1, lr, out_idx, out_val, ws,
                                     ws_bytes, stream);
+}
+
+int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float lr, int64_t k,
+                            int32_t* out_idx, float* out_val, void* stream) {
+    if (n < 0 || k < 0 || k > n || n > MAX_N) return TOPK_EF_ERR_INVALID_ARG;
+    const size_t need = topk_ef_workspace_bytes(n, k);
+    if (need == 0) return TOPK_EF_ERR_INVALID_ARG;
+    if (need > STATIC_SCRATCH_BYTES) return TOPK_EF_ERR_WORKSPACE;
+    void* ws = nullptr;
+    const int rc = static_scratch_addr(&ws);
+    if (rc != TOPK_EF_OK) return rc;
+    return topk_ef_compress(grad, residual, n, lr, k, out_idx, out_val, ws, STATIC_SCRATCH_BYTES,
+                            stream);
 }
 
 size_t gtopk_merge_workspace_bytes(int32_t P, int64_t k_in, int64_t k) {

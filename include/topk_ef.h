@@ -94,6 +94,35 @@ int topk_ef_compress(const float* grad, float* residual, int64_t n, float lr,
                      int64_t k, int32_t* out_idx, float* out_val, void* ws,
                      size_t ws_bytes, void* stream);
 
+/*
+ * topk_ef_compress_static: the same error-feedback step as topk_ef_compress,
+ * for callers that cannot allocate device memory, and so cannot provide the
+ * workspace: for instance code that runs inside a host program whose
+ * framework owns all device memory and forbids other allocations, or a
+ * latency-critical path where a cudaMalloc (which can synchronise the device)
+ * is not acceptable.  The pages have no counterpart of this entry point.
+ *
+ * The scratch it uses in place of `ws` is a fixed array of
+ * TOPK_EF_STATIC_SCRATCH_BYTES (32 MiB) inside the library's device module:
+ * every GPU on which the library is used holds it until the process exits.
+ * It allocates nothing itself: no cudaMalloc, cudaFree or allocating library
+ * routine.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ * first call before any stream capture.  Sizes whose workspace
+ * (topk_ef_workspace_bytes(n, k)) exceeds the array are rejected with
+ * TOPK_EF_ERR_WORKSPACE (32 MiB holds, e.g., n = 25.6M at k = 1% or
+ * n = 150M at k = 0.1%).  All calls share the one array and each call resets
+ * the state it needs at its start, so it keeps no result between calls; two
+ * calls whose GPU work overlaps (different streams, or different host threads
+ * without ordering) race on it and must not be issued.
+ *   Arguments and results: exactly those of topk_ef_compress, without ws and
+ *   ws_bytes.
+ */
+#define TOPK_EF_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float lr,
+                            int64_t k, int32_t* out_idx, float* out_val,
+                            void* stream);
+
 /* Workspace bytes for topk_ef_compress_batched with the same (offsets, k, T).
    offsets and k are host arrays.  Returns 0 for invalid arguments. */
 size_t topk_ef_batched_workspace_bytes(const int64_t* offsets,
