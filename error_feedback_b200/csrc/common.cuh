@@ -22,7 +22,25 @@ constexpr int D1_BITS = 11, D2_BITS = 10, D3_BITS = 10;
 constexpr int D1_BINS = 1 << D1_BITS;       // key >> 20
 constexpr int D2_BINS = 1 << D2_BITS;       // (key >> 10) & 1023
 constexpr int D3_BINS = 1 << D3_BITS;       // key & 1023
-constexpr int HIST_WORDS = D1_BINS + D1_BINS + D2_BINS + D3_BINS;  // per segment
+
+// Relative digits of a prefiltered candidate (key >= T0 of its tensor):
+//   rel = key - T0;  R1 = min(rel >> s, 4095);  R2 = rel & (2^s - 1)
+// with a per-tensor shift s <= 12; R1 = 4095 collects everything above the
+// covered range.
+constexpr int REL_BINS = 4096;
+constexpr int REL_MAX_SHIFT = 12;
+
+// Per-tensor histogram words of the compress workspace.
+constexpr int CH_R1 = 0;                        // candidates, relative digit 1
+constexpr int CH_R2 = CH_R1 + REL_BINS;         // candidates, relative digit 2
+constexpr int CH_C1 = CH_R2 + REL_BINS;         // candidates, digit 1
+constexpr int CH_D1 = CH_C1 + D1_BINS;          // residual rescan, digit 1
+constexpr int CH_D2 = CH_D1 + D1_BINS;          // digit 2 (candidates or rescan)
+constexpr int CH_D3 = CH_D2 + D2_BINS;          // digit 3
+constexpr int CHIST_WORDS = CH_D3 + D3_BINS;    // 14,336
+// Per-pair histogram words of the merge workspace.
+constexpr int MH_D1 = 0, MH_D2 = D1_BINS, MH_D3 = D1_BINS + D2_BINS;
+constexpr int MHIST_WORDS = D1_BINS + D2_BINS + D3_BINS;   // 4,096
 
 // Device status bits (ctrl.status).
 constexpr uint32_t ST_TIMEOUT = 1u;
@@ -204,6 +222,55 @@ __device__ __forceinline__ bool warp_find_bin(const uint32_t* h, int nb, uint32_
     above = __shfl_sync(0xFFFFFFFFu, rabove, src);
     cnt = __shfl_sync(0xFFFFFFFFu, rcnt, src);
     return true;
+}
+
+struct FindResult {
+    uint32_t bin, above, cnt, ok;
+};
+
+// Block-wide version of warp_find_bin over a shared-memory histogram of nb
+// bins (nb a multiple of blockDim.x, both powers of two).  Every thread of
+// the block must call it; the result is in *out after it returns.
+__device__ __forceinline__ void block_find_bin(const uint32_t* h, int nb, uint32_t rem,
+                                               uint32_t* s_red, FindResult* out) {
+    const int t = threadIdx.x;
+    const int per = nb / (int)blockDim.x;
+    const int hi = nb - t * per;   // thread 0 owns the top bins
+    const int lo = hi - per;
+    uint32_t s = 0;
+    for (int i = 0; i < per; ++i) s += h[lo + ((i + t) & (per - 1))];
+    if (t == 0) out->ok = 0;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(s, s_red, &tot);
+    if (ex < rem && ex + s >= rem) {
+        uint32_t run = ex;
+        for (int b = hi - 1; b >= lo; --b) {
+            const uint32_t c = h[b];
+            if (run + c >= rem) {
+                out->bin = (uint32_t)b;
+                out->above = run;
+                out->cnt = c;
+                out->ok = 1;
+                break;
+            }
+            run += c;
+        }
+    }
+    if (tot < rem && t == 0) {
+        out->bin = 0;
+        out->above = tot;
+        out->cnt = 0;
+    }
+    __syncthreads();
+}
+
+// Shared-memory histogram increment, aggregated over the lanes of a warp
+// that hit the same bin (the active lanes are given by `active`).
+__device__ __forceinline__ void warp_agg_inc(uint32_t* h, uint32_t bin, bool active) {
+    const uint32_t act = __ballot_sync(0xFFFFFFFFu, active);
+    if (!active) return;
+    const uint32_t peers = __match_any_sync(act, bin);
+    if ((uint32_t)(__ffs(peers) - 1) == lane_id()) atomicAdd(&h[bin], (uint32_t)__popc(peers));
 }
 
 __host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) {

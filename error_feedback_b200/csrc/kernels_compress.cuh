@@ -23,7 +23,9 @@ constexpr int TCAP_LARGE = 256;      // tensors per group
 constexpr int SAMPLE_LOG2 = 14;
 constexpr int SAMPLE_M = 1 << SAMPLE_LOG2;   // samples per sampled tensor
 constexpr int SAMPLE_THREADS = 1024;
-constexpr int SAMPLE_PER_THREAD = SAMPLE_M / SAMPLE_THREADS;
+constexpr int SAMPLE_PART = 2048;                          // samples per sampling block
+constexpr int SAMPLE_PART_PER_THREAD = SAMPLE_PART / SAMPLE_THREADS;
+constexpr int SAMPLE_PER_THREAD = SAMPLE_M / SAMPLE_THREADS;  // keys per thread in the merge
 constexpr int SAMPLE_BINS = 4096;    // key >> 19
 constexpr int K1_THREADS = 256;
 constexpr int WT = 1024;             // elements per warp tile
@@ -38,8 +40,10 @@ struct SegMeta {
     int64_t out_base;   // first output slot
     uint32_t k;
     uint32_t T0;        // prefilter threshold key (NO_KEY when k == 0)
+    uint32_t shift;     // relative digit: R1 = (key - T0) >> shift
+    uint32_t pad[3];
 };
-static_assert(sizeof(SegMeta) == 32, "SegMeta layout");
+static_assert(sizeof(SegMeta) == 48, "SegMeta layout");
 
 template <int TCAP>
 struct SetupParams {
@@ -57,63 +61,132 @@ struct SetupParams {
     int64_t off[TCAP + 1];
     int64_t out_base[TCAP];
     uint32_t k[TCAP];
-    uint32_t m[TCAP];       // samples (0: no sampling)
+    uint32_t* sample_keys;  // [T][SAMPLE_M] sampled keys
+    uint32_t* sample_done;  // [T] sampling blocks finished, cleared before the launch
+    int32_t n_sample_blocks;
+    uint32_t m[TCAP];       // samples (0: no sampling; n: every element)
     uint32_t r[TCAP];       // target rank among the samples
-    uint16_t sampled[TCAP]; // tensor of sampling block i
+    uint32_t r_hi[TCAP];    // rank of an upper estimate of the k-th key
+    uint16_t sampled[TCAP]; // i-th sampled tensor
+    uint16_t part_first[TCAP + 1];  // its first sampling block (prefix over sampled tensors)
 };
 
-// Blocks [0, n_sampled) each estimate T0 of one tensor from SAMPLE_M samples
-// of acc (256 evenly spread runs of 64 consecutive elements, so the loads
-// coalesce); the remaining blocks clear the workspace state of this call
+// The first n_sample_blocks blocks sample acc for the prefilter threshold T0
+// of the sampled tensors: every element when the tensor has at most SAMPLE_M
+// of them (then T0 is the exact k-th key), otherwise SAMPLE_M samples in 256
+// evenly spread runs of 64 consecutive elements (the loads coalesce).  Each
+// block computes SAMPLE_PART keys into the workspace; the last block of a
+// tensor to finish (a counter cleared before the launch) reads all of them
+// back from L2 and takes T0 as the r-th largest, in three histogram levels
+// (12 + 12 + 7 bits).  The shift of the relative digits is chosen so that
+// 4,095 bins of 2^shift keys above T0 reach twice past an upper estimate of
+// the k-th key.  The remaining blocks clear the workspace state of this call
 // and write the metadata of the tensors that are not sampled.
 template <int TCAP>
 __global__ void __launch_bounds__(SAMPLE_THREADS)
 setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
     __shared__ uint32_t hist[SAMPLE_BINS];
+    __shared__ uint32_t s_red[33];
+    __shared__ FindResult s_fr;
+    __shared__ int s_last;
     const int b = blockIdx.x;
     const int tid = threadIdx.x;
-    if (b < p.n_sampled) {
-        const int l = p.sampled[b];
+    if (b < p.n_sample_blocks) {
+        // which sampled tensor, which part of its samples
+        int i = 0, hi_i = p.n_sampled;
+        while (hi_i - i > 1) {
+            const int mid = (i + hi_i) >> 1;
+            if (p.part_first[mid] <= b) i = mid; else hi_i = mid;
+        }
+        const int l = p.sampled[i];
+        const int part = b - p.part_first[i];
+        const int parts = p.part_first[i + 1] - p.part_first[i];
         const int64_t off = p.off[l];
         const int64_t n = p.off[l + 1] - off;
         const uint32_t m = p.m[l];
-        for (int i = tid; i < SAMPLE_BINS; i += blockDim.x) hist[i] = 0;
+        const bool full = (int64_t)m == n;
+        uint32_t* keys = p.sample_keys + (size_t)l * SAMPLE_M;
+#pragma unroll
+        for (int u = 0; u < SAMPLE_PART_PER_THREAD; ++u) {
+            const uint32_t s = (uint32_t)(part * SAMPLE_PART + u * SAMPLE_THREADS + tid);
+            if (s < m) {
+                // every element, or 256 runs of 64 consecutive elements
+                const int64_t pos = full ? off + s : off + (((int64_t)(s >> 6) * n) >> 8) + (s & 63);
+                keys[s] = key_of(__fmaf_rn(p.lr, __ldg(p.grad + pos), __ldg(p.resid + pos)));
+            }
+        }
+        // the last sampling block of the tensor computes the quantile
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(&p.sample_done[l], 1u) == (uint32_t)(parts - 1);
+        __syncthreads();
+        if (!s_last) return;
+        __threadfence();
+        for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
         __syncthreads();
         uint32_t key[SAMPLE_PER_THREAD];
 #pragma unroll
         for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
             const uint32_t s = (uint32_t)(u * SAMPLE_THREADS + tid);
-            key[u] = NO_KEY;
-            if (s < m) {
-                // 256 chunks of 64 consecutive elements, evenly spread
-                const int64_t pos = off + (((int64_t)(s >> 6) * n) >> 8) + (s & 63);
-                const float a = __fmaf_rn(p.lr, __ldg(p.grad + pos), __ldg(p.resid + pos));
-                key[u] = key_of(a);
-            }
+            key[u] = s < m ? __ldcg(keys + s) : NO_KEY;
         }
+        // level 1: key >> 19
 #pragma unroll
         for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
             if (key[u] != NO_KEY) atomicAdd(&hist[key[u] >> 19], 1u);
         __syncthreads();
-        if (tid < 32) {
-            uint32_t bin, above, cnt;
-            warp_find_bin(hist, SAMPLE_BINS, p.r[l], bin, above, cnt);
-            if (tid == 0) {
-                SegMeta sm;
-                sm.off = off;
-                sm.n = n;
-                sm.out_base = p.out_base[l];
-                sm.k = p.k[l];
-                // never above 0x7F800001: then "raw |x| bits >= T0" and "key >= T0"
-                // agree for NaN too (lowering T0 only adds candidates)
-                sm.T0 = min(bin << 19, 0x7F800001u);
-                p.meta[l] = sm;
-            }
+        block_find_bin(hist, SAMPLE_BINS, p.r[l], s_red, &s_fr);
+        const uint32_t ok1 = s_fr.ok, b1 = s_fr.bin;
+        uint32_t rem = p.r[l] - s_fr.above;
+        __syncthreads();
+        block_find_bin(hist, SAMPLE_BINS, p.r_hi[l], s_red, &s_fr);
+        const uint32_t bhi = s_fr.ok ? s_fr.bin : b1;
+        // level 2: bits 18..7 of the keys in bin b1
+        __syncthreads();
+        for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+            if (key[u] != NO_KEY && (key[u] >> 19) == b1) atomicAdd(&hist[(key[u] >> 7) & 4095u], 1u);
+        __syncthreads();
+        block_find_bin(hist, SAMPLE_BINS, rem, s_red, &s_fr);
+        const uint32_t ok2 = s_fr.ok, b2 = s_fr.bin;
+        rem -= s_fr.above;
+        // level 3: bits 6..0 of the keys in that sub-bin
+        __syncthreads();
+        for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
+        __syncthreads();
+        const uint32_t pre = (b1 << 12) | b2;
+#pragma unroll
+        for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+            if (key[u] != NO_KEY && (key[u] >> 7) == pre) atomicAdd(&hist[key[u] & 127u], 1u);
+        __syncthreads();
+        block_find_bin(hist, SAMPLE_BINS, rem, s_red, &s_fr);
+        const uint32_t ok3 = s_fr.ok, b3 = s_fr.bin;
+        if (tid == 0) {
+            uint32_t T0 = 0;
+            if (ok1 && ok2 && ok3) T0 = (pre << 7) | b3;
+            // never above 0x7F800001: then "raw |x| bits >= T0" and "key >= T0"
+            // agree for NaN too (lowering T0 only adds candidates)
+            T0 = min(T0, 0x7F800001u);
+            const uint64_t hi = ((uint64_t)(bhi + 1) << 19);
+            const uint64_t d = hi > T0 ? hi - T0 : 0;
+            uint32_t sh = 0;
+            while (sh < (uint32_t)REL_MAX_SHIFT && ((uint64_t)(REL_BINS - 1) << sh) <= 2 * d) ++sh;
+            SegMeta sm;
+            memset(&sm, 0, sizeof(sm));
+            sm.off = off;
+            sm.n = n;
+            sm.out_base = p.out_base[l];
+            sm.k = p.k[l];
+            sm.T0 = T0;
+            sm.shift = sh;
+            p.meta[l] = sm;
         }
         return;
     }
-    const int zb = b - p.n_sampled;
-    const int nz = gridDim.x - p.n_sampled;
+    const int zb = b - p.n_sample_blocks;
+    const int nz = gridDim.x - p.n_sample_blocks;
     if (zb == 0) {
         if (tid == 0) {
             Ctrl c;
@@ -125,11 +198,13 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
         for (int l = tid; l < p.T; l += blockDim.x) {
             if (p.m[l] != 0) continue;
             SegMeta sm;
+            memset(&sm, 0, sizeof(sm));
             sm.off = p.off[l];
             sm.n = p.off[l + 1] - p.off[l];
             sm.out_base = p.out_base[l];
             sm.k = p.k[l];
             sm.T0 = p.k[l] == 0 ? NO_KEY : 0u;
+            sm.shift = REL_MAX_SHIFT;
             p.meta[l] = sm;
         }
     }
@@ -151,7 +226,7 @@ struct StreamParams {
     uint32_t* wt_count;     // [num_wt] candidates of each warp tile (exact)
     uint32_t* st_idx;       // [num_wt][WT_CAP] staged candidates, index order
     float* st_val;
-    uint32_t* hist;         // [T][HIST_WORDS]; candidate digit 1 at offset 0
+    uint32_t* hist;         // [T][CHIST_WORDS]: candidate R1 at CH_R1, digit 1 at CH_C1
     uint32_t* bound_before; // [T]: candidates of the warp tile holding off[l] below off[l]
 };
 
@@ -175,49 +250,169 @@ __device__ __forceinline__ int lower_bound_off(const int64_t* off, int T, int64_
     return lo;
 }
 
+struct StreamShared {
+    int64_t off[TCAP_LARGE + 1];
+    uint32_t T0[TCAP_LARGE];
+    uint32_t sh[TCAP_LARGE];
+    uint32_t r1[REL_BINS];     // one tensor: candidate histograms in shared memory
+    uint32_t c1[D1_BINS];
+};
+
+// General warp tile: a partial last tile, a tile that spans tensors, or
+// unaligned inputs.  Computes acc, stores it, returns the candidate flags
+// (bit 4j + v for element base + 128 j + 4 lane + v).
+template <bool VEC>
+__device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, const StreamShared& S,
+                                                     int64_t base, int l_lo, int l_hi) {
+    const uint32_t lane = lane_id();
+    uint32_t flags = 0;
+    for (int j = 0; j < WT_VECS; ++j) {
+        const int64_t e = base + j * 128 + lane * 4;
+        float a[4];
+        if (VEC && e + 3 < p.N) {
+            const float4 gv = ld_stream(reinterpret_cast<const float4*>(p.grad + e));
+            const float4 rv = ld_stream(reinterpret_cast<const float4*>(p.resid + e));
+            a[0] = __fmaf_rn(p.lr, gv.x, rv.x);
+            a[1] = __fmaf_rn(p.lr, gv.y, rv.y);
+            a[2] = __fmaf_rn(p.lr, gv.z, rv.z);
+            a[3] = __fmaf_rn(p.lr, gv.w, rv.w);
+            st_stream(reinterpret_cast<float4*>(p.resid + e), make_float4(a[0], a[1], a[2], a[3]));
+        } else {
+            for (int v = 0; v < 4; ++v) {
+                a[v] = 0.f;
+                if (e + v < p.N) {
+                    a[v] = __fmaf_rn(p.lr, __ldcs(p.grad + e + v), __ldcs(p.resid + e + v));
+                    __stcs(p.resid + e + v, a[v]);
+                }
+            }
+        }
+        for (int v = 0; v < 4; ++v) {
+            if (e + v >= p.N) continue;
+            int l = l_lo;
+            while (l < l_hi && S.off[l + 1] <= e + v) ++l;
+            if (key_of(a[v]) >= S.T0[l]) flags |= 1u << (j * 4 + v);
+        }
+    }
+    return flags;
+}
+
+// Rare path of a warp tile with candidates: count them, stage them in index
+// order, add them to the candidate histograms (acc is read back from the
+// residual the warp has just written), and record the warp tile's count.
+__device__ __noinline__ void stream_tile_candidates(const StreamParams& p, StreamShared& S,
+                                                    uint32_t w, int64_t base, int l_lo, int l_hi,
+                                                    uint32_t flags, bool flat) {
+    const uint32_t lane = lane_id();
+    const uint32_t cnt = warp_sum((uint32_t)__popc(flags));
+    if (lane == 0) p.wt_count[w] = cnt;
+    uint32_t before = 0;   // candidates of earlier vectors
+    for (int j = 0; j < WT_VECS; ++j) {
+        const uint32_t fj = (flags >> (4 * j)) & 0xFu;
+        if (!__any_sync(0xFFFFFFFFu, fj != 0)) continue;
+        const uint32_t c = __popc(fj);
+        const uint32_t incl = warp_incl_scan(c);
+        uint32_t pos = before + incl - c;
+        const int64_t e = base + j * 128 + lane * 4;
+        for (int v = 0; v < 4; ++v) {
+            if (!((fj >> v) & 1u)) continue;
+            const float a = __ldcg(p.resid + e + v);
+            if (cnt <= WT_CAP) {
+                p.st_idx[(size_t)w * WT_CAP + pos] = (uint32_t)(e + v);
+                p.st_val[(size_t)w * WT_CAP + pos] = a;
+            }
+            const uint32_t key = key_of(a);
+            int l = l_lo;
+            while (l < l_hi && S.off[l + 1] <= e + v) ++l;
+            const uint32_t rb = min((key - S.T0[l]) >> S.sh[l], (uint32_t)(REL_BINS - 1));
+            if (flat) {
+                atomicAdd(&S.r1[rb], 1u);
+                atomicAdd(&S.c1[key >> 20], 1u);
+            } else {
+                atomicAdd(&p.hist[(size_t)l * CHIST_WORDS + CH_R1 + rb], 1u);
+                atomicAdd(&p.hist[(size_t)l * CHIST_WORDS + CH_C1 + (key >> 20)], 1u);
+            }
+            ++pos;
+        }
+        before += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+}
+
+// Tensors that start inside warp tile [base, tend): candidates below each start.
+__device__ __noinline__ void stream_tile_bounds(const StreamParams& p, const StreamShared& S,
+                                                int64_t base, int64_t tend, uint32_t flags) {
+    const uint32_t lane = lane_id();
+    const int T = p.T;
+    const int lb = max(1, lower_bound_off(S.off, T, base));
+    const int ub = min(T, lower_bound_off(S.off, T, tend));
+    for (int l = lb; l < ub; ++l) {
+        const int64_t bound = S.off[l];
+        uint32_t c = 0;
+        for (int j = 0; j < WT_VECS; ++j) {
+            const int64_t e = base + j * 128 + lane * 4;
+            for (int v = 0; v < 4; ++v) c += ((flags >> (j * 4 + v)) & 1u) && (e + v < bound);
+        }
+        c = warp_sum(c);
+        if (lane == 0) p.bound_before[l] = c;
+    }
+}
+
 // The fused streaming pass, the only full sweep of the step:
 //   acc = fmaf(lr, grad, residual) written back to residual;
 //   candidates (key >= T0 of the element's tensor) staged per warp tile in
 //   index order (at most WT_CAP; the count is always exact);
-//   digit-1 histogram of the candidates per tensor.
+//   histograms of the candidates' relative digit 1 and digit 1 per tensor.
 // Each warp owns whole 1,024-element warp tiles (grid-stride), so warps never
 // wait for one another: the global order of the candidates is rebuilt by the
-// select kernel from the per-warp-tile counts.
+// select kernel from the per-warp-tile counts.  The loop over full tiles of
+// one tensor is kept small; everything else is out of line.
 template <bool VEC>
 __global__ void __launch_bounds__(K1_THREADS, 3)
 stream_kernel(const StreamParams p) {
-    __shared__ int64_t s_off[TCAP_LARGE + 1];
-    __shared__ uint32_t s_T0[TCAP_LARGE];
-    __shared__ uint32_t s_h1[D1_BINS];
-
+    __shared__ StreamShared S;
     const int tid = threadIdx.x;
     const uint32_t lane = lane_id();
     const int T = p.T;
     const bool flat = (T == 1);
     for (int l = tid; l < T; l += blockDim.x) {
-        s_off[l] = p.meta[l].off;
-        s_T0[l] = p.meta[l].T0;
+        S.off[l] = p.meta[l].off;
+        S.T0[l] = p.meta[l].T0;
+        S.sh[l] = p.meta[l].shift;
     }
-    if (tid == 0) s_off[T] = p.N;
-    if (flat)
-        for (int i = tid; i < D1_BINS; i += blockDim.x) s_h1[i] = 0;
+    if (tid == 0) S.off[T] = p.N;
+    if (flat) {
+        for (int i = tid; i < REL_BINS; i += blockDim.x) S.r1[i] = 0;
+        for (int i = tid; i < D1_BINS; i += blockDim.x) S.c1[i] = 0;
+    }
     __syncthreads();
 
+    // Warp tiles are handed out statically for all but the last rounds, then
+    // by ticket, so that no warp is left with a whole extra round at the end.
     const uint32_t warps = blockDim.x >> 5;
     const uint32_t gw = blockIdx.x * warps + warp_id();
     const uint32_t GW = gridDim.x * warps;
-    for (uint32_t w = gw; w < p.num_wt; w += GW) {
+    const uint32_t R = p.num_wt / GW >= 2 ? p.num_wt / GW - 1 : 0;   // static rounds
+    const float lr = p.lr;
+    uint32_t w;
+    if (R > 0) {
+        w = gw;
+    } else {
+        uint32_t t = 0;
+        if (lane == 0) t = atomicAdd(&p.ctrl->tile_ticket, 1u);
+        w = R * GW + __shfl_sync(0xFFFFFFFFu, t, 0);
+    }
+    for (uint32_t round = 0; w < p.num_wt; ++round) {
+        // next tile: static, or a ticket fetched now and read after this tile
+        uint32_t ticket = 0;
+        const bool stat_next = round + 1 < R;
+        if (!stat_next && lane == 0) ticket = atomicAdd(&p.ctrl->tile_ticket, 1u);
         const int64_t base = (int64_t)w * WT;
         const int64_t tend = min(base + (int64_t)WT, p.N);
-        const int l_lo = flat ? 0 : seg_of(s_off, T, base);
-        const int l_hi = flat ? 0 : seg_of(s_off, T, tend - 1);
-        const bool uniform = (l_lo == l_hi);
-        const uint32_t T0u = s_T0[l_lo];
-
-        float r[WT_VECS][4];
+        const int l_lo = flat ? 0 : seg_of(S.off, T, base);
+        const int l_hi = flat ? 0 : seg_of(S.off, T, tend - 1);
         uint32_t flags = 0;
-        if (VEC && uniform && tend - base == WT) {
+        if (VEC && l_lo == l_hi && tend - base == WT) {
             // full warp tile inside one tensor: 128-bit loads, no bounds checks
+            const uint32_t T0 = S.T0[l_lo];
             const float4* g4 = reinterpret_cast<const float4*>(p.grad + base) + lane;
             float4* r4 = reinterpret_cast<float4*>(p.resid + base) + lane;
             float4 gv[WT_VECS], rv[WT_VECS];
@@ -229,126 +424,33 @@ stream_kernel(const StreamParams p) {
 #pragma unroll
             for (int j = 0; j < WT_VECS; ++j) {
                 float4 a;
-                a.x = __fmaf_rn(p.lr, gv[j].x, rv[j].x);
-                a.y = __fmaf_rn(p.lr, gv[j].y, rv[j].y);
-                a.z = __fmaf_rn(p.lr, gv[j].z, rv[j].z);
-                a.w = __fmaf_rn(p.lr, gv[j].w, rv[j].w);
+                a.x = __fmaf_rn(lr, gv[j].x, rv[j].x);
+                a.y = __fmaf_rn(lr, gv[j].y, rv[j].y);
+                a.z = __fmaf_rn(lr, gv[j].z, rv[j].z);
+                a.w = __fmaf_rn(lr, gv[j].w, rv[j].w);
                 st_stream(r4 + 32 * j, a);
-                r[j][0] = a.x; r[j][1] = a.y; r[j][2] = a.z; r[j][3] = a.w;
-                flags |= (uint32_t)((__float_as_uint(a.x) & KEY_MASK) >= T0u) << (4 * j);
-                flags |= (uint32_t)((__float_as_uint(a.y) & KEY_MASK) >= T0u) << (4 * j + 1);
-                flags |= (uint32_t)((__float_as_uint(a.z) & KEY_MASK) >= T0u) << (4 * j + 2);
-                flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0u) << (4 * j + 3);
+                flags |= (uint32_t)((__float_as_uint(a.x) & KEY_MASK) >= T0) << (4 * j);
+                flags |= (uint32_t)((__float_as_uint(a.y) & KEY_MASK) >= T0) << (4 * j + 1);
+                flags |= (uint32_t)((__float_as_uint(a.z) & KEY_MASK) >= T0) << (4 * j + 2);
+                flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0) << (4 * j + 3);
             }
         } else {
-            float g[WT_VECS][4];
-#pragma unroll
-            for (int j = 0; j < WT_VECS; ++j) {
-                const int64_t e = base + j * 128 + lane * 4;
-                if (VEC && e + 3 < p.N) {
-                    const float4 gv = ld_stream(reinterpret_cast<const float4*>(p.grad + e));
-                    const float4 rv = ld_stream(reinterpret_cast<const float4*>(p.resid + e));
-                    g[j][0] = gv.x; g[j][1] = gv.y; g[j][2] = gv.z; g[j][3] = gv.w;
-                    r[j][0] = rv.x; r[j][1] = rv.y; r[j][2] = rv.z; r[j][3] = rv.w;
-                } else {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        g[j][v] = 0.f;
-                        r[j][v] = 0.f;
-                        if (e + v < p.N) {
-                            g[j][v] = __ldcs(p.grad + e + v);
-                            r[j][v] = __ldcs(p.resid + e + v);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < WT_VECS; ++j) {
-                const int64_t e = base + j * 128 + lane * 4;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float a = __fmaf_rn(p.lr, g[j][v], r[j][v]);
-                    r[j][v] = a;
-                    if (e + v < p.N) {
-                        uint32_t T0 = T0u;
-                        if (!uniform) {
-                            int l = l_lo;
-                            while (l < l_hi && s_off[l + 1] <= e + v) ++l;
-                            T0 = s_T0[l];
-                        }
-                        if (key_of(a) >= T0) flags |= 1u << (j * 4 + v);
-                    }
-                }
-                if (VEC && e + 3 < p.N) {
-                    st_stream(reinterpret_cast<float4*>(p.resid + e),
-                              make_float4(r[j][0], r[j][1], r[j][2], r[j][3]));
-                } else {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        if (e + v < p.N) __stcs(p.resid + e + v, r[j][v]);
-                }
-            }
+            flags = stream_tile_general<VEC>(p, S, base, l_lo, l_hi);
         }
-
-        // candidates of the warp tile, in index order (vector j, lane, element v)
-        const uint32_t any = __ballot_sync(0xFFFFFFFFu, flags != 0);
-        const uint32_t cnt = any ? warp_sum((uint32_t)__popc(flags)) : 0u;
-        if (lane == 0) p.wt_count[w] = cnt;
-        if (cnt) {
-            uint32_t before = 0;   // candidates of earlier vectors
-#pragma unroll
-            for (int j = 0; j < WT_VECS; ++j) {
-                const uint32_t fj = (flags >> (4 * j)) & 0xFu;
-                if (!__any_sync(0xFFFFFFFFu, fj != 0)) continue;
-                const uint32_t c = __popc(fj);
-                const uint32_t incl = warp_incl_scan(c);
-                uint32_t pos = before + incl - c;
-                const int64_t e = base + j * 128 + lane * 4;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (!((fj >> v) & 1u)) continue;
-                    if (cnt <= WT_CAP) {
-                        p.st_idx[(size_t)w * WT_CAP + pos] = (uint32_t)(e + v);
-                        p.st_val[(size_t)w * WT_CAP + pos] = r[j][v];
-                    }
-                    const uint32_t bin = key_of(r[j][v]) >> 20;
-                    if (flat) {
-                        atomicAdd(&s_h1[bin], 1u);
-                    } else {
-                        int l = l_lo;
-                        if (!uniform)
-                            while (l < l_hi && s_off[l + 1] <= e + v) ++l;
-                        atomicAdd(&p.hist[(size_t)l * HIST_WORDS + bin], 1u);
-                    }
-                    ++pos;
-                }
-                before += __shfl_sync(0xFFFFFFFFu, incl, 31);
-            }
+        if (__any_sync(0xFFFFFFFFu, flags != 0)) {
+            stream_tile_candidates(p, S, w, base, l_lo, l_hi, flags, flat);
+        } else if (lane == 0) {
+            p.wt_count[w] = 0;
         }
-
-        // tensors that start inside this warp tile: candidates below the start
-        if (!flat) {
-            const int lb = max(1, lower_bound_off(s_off, T, base));
-            const int ub = min(T, lower_bound_off(s_off, T, tend));
-            for (int l = lb; l < ub; ++l) {
-                const int64_t bound = s_off[l];
-                uint32_t c = 0;
-#pragma unroll
-                for (int j = 0; j < WT_VECS; ++j) {
-                    const int64_t e = base + j * 128 + lane * 4;
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        c += ((flags >> (j * 4 + v)) & 1u) && (e + v < bound);
-                }
-                c = warp_sum(c);
-                if (lane == 0) p.bound_before[l] = c;
-            }
-        }
+        if (!flat) stream_tile_bounds(p, S, base, tend, flags);
+        w = stat_next ? w + GW : R * GW + __shfl_sync(0xFFFFFFFFu, ticket, 0);
     }
     if (flat) {
         __syncthreads();
+        for (int i = tid; i < REL_BINS; i += blockDim.x)
+            if (S.r1[i]) atomicAdd(&p.hist[CH_R1 + i], S.r1[i]);
         for (int i = tid; i < D1_BINS; i += blockDim.x)
-            if (s_h1[i]) atomicAdd(&p.hist[i], s_h1[i]);
+            if (S.c1[i]) atomicAdd(&p.hist[CH_C1 + i], S.c1[i]);
     }
 }
 

@@ -94,7 +94,7 @@ struct MergeRoundParams {
     int64_t mcap;               // merged positions per pair
     uint32_t* m_idx;            // [np][mcap]
     float* m_val;
-    uint32_t* hist;             // pair p: digit-1 histogram at p * HIST_WORDS
+    uint32_t* hist;             // pair p: digit-1 histogram at p * MHIST_WORDS
     uint32_t* live;             // [np]
 };
 
@@ -203,16 +203,21 @@ merge_round_kernel(const MergeRoundParams p) {
     const int span = (int)(d1 - d0);
     uint32_t live = 0;
     const int dl = tid * MG_PER_THREAD;
+    // every lane runs the same MG_PER_THREAD steps (the histogram update is
+    // aggregated across the warp); lanes past the span do nothing
+    int ia = 0, ib = 0;
     if (dl < span) {
-        int ia = local_merge_path(sAi + 1, la, sBi, lb, dl);
-        int ib = dl - ia;
+        ia = local_merge_path(sAi + 1, la, sBi, lb, dl);
+        ib = dl - ia;
+    }
 #pragma unroll
-        for (int u = 0; u < MG_PER_THREAD; ++u) {
-            const int pos = dl + u;
-            if (pos >= span) break;
+    for (int u = 0; u < MG_PER_THREAD; ++u) {
+        const int pos = dl + u;
+        const bool valid = pos < span;
+        uint32_t oi = DEAD;
+        float ov = 0.f;
+        if (valid) {
             const int64_t d = d0 + pos;
-            uint32_t oi;
-            float ov;
             const bool takeA = ia < la && (ib >= lb || sAi[1 + ia] <= sBi[ib]);
             if (takeA) {
                 oi = sAi[1 + ia];
@@ -237,11 +242,9 @@ merge_round_kernel(const MergeRoundParams p) {
             }
             Mi[d] = oi;
             Mv[d] = oi == DEAD ? 0.f : ov;
-            if (oi != DEAD) {
-                ++live;
-                atomicAdd(&s_h1[key_of(ov) >> 20], 1u);
-            }
+            if (oi != DEAD) ++live;
         }
+        if (valid && oi != DEAD) atomicAdd(&s_h1[key_of(ov) >> 20], 1u);
     }
     // the block that ends the merged list clears the tail of the segment
     if (d1 == ab)
@@ -251,7 +254,7 @@ merge_round_kernel(const MergeRoundParams p) {
         }
     const uint32_t tl = block_sum(live, s_red);
     if (tid == 0 && tl) atomicAdd(&p.live[pair], tl);
-    uint32_t* h = p.hist + (size_t)pair * HIST_WORDS;
+    uint32_t* h = p.hist + (size_t)pair * MHIST_WORDS + MH_D1;
     for (int i = tid; i < D1_BINS; i += blockDim.x)
         if (s_h1[i]) atomicAdd(&h[i], s_h1[i]);
 }

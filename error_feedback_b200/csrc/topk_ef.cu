@@ -30,7 +30,6 @@ thread_local int t_last_cuda_error = 0;
 std::atomic<int> g_test_flags{0};
 
 constexpr int64_t MAX_N = 2147483647LL;
-constexpr int64_t SMALL_N = 65536;     // tensors up to this size are not sampled
 constexpr int SLOT_MAX = 2048;         // select grid never exceeds this
 constexpr size_t ALIGN = 256;
 constexpr int MAX_MERGE_P = 2 * SEG_MAX;   // pairs per round <= SEG_MAX
@@ -117,7 +116,7 @@ int device_facts(DevFacts* out) {
 // threshold among them, and the candidate capacity reserved for it.
 struct TensorPlan {
     int64_t off, n, out_base;
-    uint32_t k, m, r;
+    uint32_t k, m, r, r_hi;
     int64_t cap;
 };
 
@@ -129,22 +128,30 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
     t.k = (uint32_t)k;
     t.m = 0;
     t.r = 0;
+    t.r_hi = 0;
     if (k == 0) {
         t.cap = 0;
-    } else if (n <= SMALL_N) {
+    } else if (n <= SAMPLE_M) {
+        // every element is sampled: T0 is the exact k-th key
+        t.m = (uint32_t)n;
+        t.r = (uint32_t)k;
+        t.r_hi = (uint32_t)k;
         t.cap = n;
     } else {
-        // Expected sample count above the k-th key: ks = k * m / n.  Aim the
-        // threshold at ks + 6 sqrt(ks) + 16 samples so that it is below the
-        // k-th key unless the sample is far from typical.
+        // Expected sample count above the k-th key: ks = k * m / n.  Put the
+        // threshold at the sample of rank ks + 4 sqrt(ks) + 4, below the k-th
+        // key unless the sample is far from typical (then the select kernel
+        // rescans the residual); rank ks - 3 sqrt(ks) - 2 estimates the k-th
+        // key from above.
         const double m = (double)SAMPLE_M;
         const double ks = (double)k * m / (double)n;
-        const double r = std::ceil(ks + 6.0 * std::sqrt(ks) + 16.0);
+        const double r = std::ceil(ks + 4.0 * std::sqrt(ks) + 4.0);
         if (r >= m) {
             t.cap = n;
         } else {
             t.m = (uint32_t)SAMPLE_M;
             t.r = (uint32_t)r;
+            t.r_hi = (uint32_t)std::max(1.0, std::floor(ks - 3.0 * std::sqrt(ks) - 2.0));
             const double e = 2.5 * r * (double)n / m + 4096.0;
             t.cap = std::min<int64_t>(n, (int64_t)std::ceil(e));
         }
@@ -154,8 +161,8 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
 
 // Workspace layout of one compress group (<= TCAP_LARGE tensors).
 struct CLayout {
-    size_t ctrl, meta, zero_begin, cand_start, hist, zero_end, bound_before, wt_count, st_idx,
-        st_val, slots, cand_idx, cand_val, total;
+    size_t ctrl, meta, sample_done, zero_begin, cand_start, hist, zero_end, bound_before, wt_count,
+        st_idx, st_val, sample_keys, slots, cand_idx, cand_val, total;
     int64_t cap;
     uint32_t num_wt;
 };
@@ -172,11 +179,13 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + sizeof(Ctrl));
     L.meta = o;
     o = align_up(o + T * sizeof(SegMeta));
+    L.sample_done = o;
+    o = align_up(o + T * sizeof(uint32_t));
     L.zero_begin = o;
     L.cand_start = o;
     o = align_up(o + (T + 1) * sizeof(int64_t));
     L.hist = o;
-    o = align_up(o + T * HIST_WORDS * sizeof(uint32_t));
+    o = align_up(o + T * CHIST_WORDS * sizeof(uint32_t));
     L.zero_end = o;
     L.bound_before = o;
     o = align_up(o + (T + 1) * sizeof(uint32_t));
@@ -186,6 +195,8 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(uint32_t));
     L.st_val = o;
     o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(float));
+    L.sample_keys = o;
+    o = align_up(o + T * (size_t)SAMPLE_M * sizeof(uint32_t));
     L.slots = o;
     o = align_up(o + SLOT_MAX * sizeof(Slot));
     L.cand_idx = o;
@@ -252,7 +263,9 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
     p.meta = reinterpret_cast<SegMeta*>(ws + L.meta);
     p.zero_ptr = reinterpret_cast<uint4*>(ws + L.zero_begin);
     p.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
-    int ns = 0;
+    p.sample_keys = reinterpret_cast<uint32_t*>(ws + L.sample_keys);
+    p.sample_done = reinterpret_cast<uint32_t*>(ws + L.sample_done);
+    int ns = 0, blocks = 0;
     for (int l = 0; l < T; ++l) {
         const TensorPlan& t = g.plans[l];
         p.off[l] = t.off;
@@ -260,13 +273,25 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
         p.k[l] = t.k;
         p.m[l] = force_t0_zero ? 0u : t.m;
         p.r[l] = t.r;
-        if (p.m[l]) p.sampled[ns++] = (uint16_t)l;
+        p.r_hi[l] = t.r_hi;
+        if (p.m[l]) {
+            p.sampled[ns] = (uint16_t)l;
+            p.part_first[ns] = (uint16_t)blocks;
+            blocks += (int)((p.m[l] + SAMPLE_PART - 1) / SAMPLE_PART);
+            ++ns;
+        }
     }
+    p.part_first[ns] = (uint16_t)blocks;
     p.off[T] = g.N;
     p.n_sampled = ns;
+    p.n_sample_blocks = blocks;
+    if (blocks) {
+        cudaError_t e = cudaMemsetAsync(ws + L.sample_done, 0, T * sizeof(uint32_t), st);
+        if (e != cudaSuccess) return e;
+    }
     const uint64_t per_block = (uint64_t)ZERO_THREADS * 8;
     const int nz = (int)std::max<uint64_t>(1, std::min<uint64_t>(148, (p.zero_vec4 + per_block - 1) / per_block));
-    setup_kernel<TCAP><<<ns + nz, SAMPLE_THREADS, 0, st>>>(p);
+    setup_kernel<TCAP><<<blocks + nz, SAMPLE_THREADS, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -421,7 +446,7 @@ MLayout merge_layout(int32_t P, int64_t k_in, int64_t k) {
     o = align_up(o + 148 * sizeof(uint32_t));
     L.zero_begin = o;
     L.hist = o;
-    o = align_up(o + (size_t)hsegs * HIST_WORDS * sizeof(uint32_t));
+    o = align_up(o + (size_t)hsegs * MHIST_WORDS * sizeof(uint32_t));
     L.live = o;
     o = align_up(o + (size_t)hsegs * sizeof(uint32_t));
     L.zero_end = o;
@@ -624,7 +649,7 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
         mp.mcap = L.mcap[r];
         mp.m_idx = m_idx;
         mp.m_val = m_val;
-        mp.hist = hist + (size_t)L.pbase[r] * HIST_WORDS;
+        mp.hist = hist + (size_t)L.pbase[r] * MHIST_WORDS;
         mp.live = live + L.pbase[r];
         dim3 grid((unsigned)ceil_div64(L.mcap[r], MG_D), (unsigned)L.np[r]);
         trace_before(st, "merge_round_kernel");
