@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(ctypes.c_char_p), ctypes.c_int,
                                          ctypes.POINTER(ctypes.c_int)]
         L.topk_ef_trace_read.restype = ctypes.c_int
+        L.topk_ef_trace_only.argtypes = [ctypes.c_char_p, ctypes.c_int]
+        L.topk_ef_trace_only.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -265,8 +267,9 @@ def topk_ef_path_info(ws, stream=None) -> dict:
 
 
 def topk_ef_phase_times(ws, stream=None) -> list:
-    """Select kernel phase end times (ns from its start; -1: phase not run)."""
-    ns = (ctypes.c_int64 * 8)()
+    """Diagnostic timestamps of the last compress call on ws (12 values, ns;
+    -1: step not run): select kernel phases, then the sampling block."""
+    ns = (ctypes.c_int64 * 12)()
     _check(lib().topk_ef_phase_times(ws.data_ptr(), _stream(stream), ns), "topk_ef_phase_times")
     return [int(x) for x in ns]
 
@@ -275,9 +278,13 @@ def topk_ef_set_test_flags(flags: int) -> int:
     return int(lib().topk_ef_set_test_flags(int(flags)))
 
 
-def topk_ef_trace_enable(on: bool = True) -> None:
-    """Record CUDA events around every kernel the library launches."""
-    _check(lib().topk_ef_trace_enable(1 if on else 0), "topk_ef_trace_enable")
+def topk_ef_trace_enable(on: bool = True, only: str | None = None, every: int = 1) -> None:
+    """Record CUDA events around every kernel the library launches, or only
+    around the launches of kernel `only`, every `every`-th of them."""
+    L = lib()
+    _check(L.topk_ef_trace_only(only.encode() if only else None, int(every)),
+           "topk_ef_trace_only")
+    _check(L.topk_ef_trace_enable(1 if on else 0), "topk_ef_trace_enable")
 
 
 def topk_ef_trace_read() -> list:

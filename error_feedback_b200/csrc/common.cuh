@@ -32,12 +32,11 @@ constexpr int REL_MAX_SHIFT = 12;
 
 // Per-tensor histogram words of the compress workspace.
 constexpr int CH_R1 = 0;                        // candidates, relative digit 1
-constexpr int CH_R2 = CH_R1 + REL_BINS;         // candidates, relative digit 2
-constexpr int CH_C1 = CH_R2 + REL_BINS;         // candidates, digit 1
-constexpr int CH_D1 = CH_C1 + D1_BINS;          // residual rescan, digit 1
-constexpr int CH_D2 = CH_D1 + D1_BINS;          // digit 2 (candidates or rescan)
-constexpr int CH_D3 = CH_D2 + D2_BINS;          // digit 3
-constexpr int CHIST_WORDS = CH_D3 + D3_BINS;    // 14,336
+constexpr int CH_R2 = CH_R1 + REL_BINS;         // candidates in the k-th key's R1 bin, R2
+constexpr int CH_D1 = CH_R2 + REL_BINS;         // residual rescan, digit 1
+constexpr int CH_D2 = CH_D1 + D1_BINS;          // residual rescan, digit 2
+constexpr int CH_D3 = CH_D2 + D2_BINS;          // residual rescan, digit 3
+constexpr int CHIST_WORDS = CH_D3 + D3_BINS;    // 12,288
 // Per-pair histogram words of the merge workspace.
 constexpr int MH_D1 = 0, MH_D2 = D1_BINS, MH_D3 = D1_BINS + D2_BINS;
 constexpr int MHIST_WORDS = D1_BINS + D2_BINS + D3_BINS;   // 4,096
@@ -59,7 +58,7 @@ struct Ctrl {
     uint64_t cand_total;    // candidates kept by the prefilter
     uint64_t cap;           // candidate capacity
     uint32_t kernels;       // kernels the call launched
-    uint32_t pad0;
+    uint32_t r2_path;       // compress: a tensor's k-th bin was too full for its entry list
     uint32_t merge_bar[32]; // grid barrier counters, one per merge round
     uint32_t pad1[6];
     uint64_t t_phase[8];    // select kernel: globaltimer at each phase (block 0)

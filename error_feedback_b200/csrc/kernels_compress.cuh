@@ -6,8 +6,8 @@
 // ABSTRACT) computes acc = fmaf(lr, grad, residual), keeps the k entries of
 // largest |acc| and leaves the rest in memory.  The only pass over the full
 // tensor is the streaming kernel below: it reads grad and residual once,
-// writes acc back into residual, and stages every element whose key reaches
-// a prefilter threshold T0 as a candidate.  The exact top-k is then found
+// writes acc back into residual, and records where the elements whose key
+// reaches a prefilter threshold T0 (the candidates) are.  The exact top-k is then found
 // among the candidates (select kernel).  T0 comes from a strided sample; if
 // it turns out too high (fewer than k candidates) or too low (candidate
 // capacity exceeded) the select kernel rescans the residual instead, so the
@@ -20,17 +20,16 @@ namespace tke {
 
 constexpr int TCAP_SMALL = 8;        // setup parameter block for T <= 8
 constexpr int TCAP_LARGE = 256;      // tensors per group
-constexpr int SAMPLE_LOG2 = 14;
+constexpr int SAMPLE_LOG2 = 13;
 constexpr int SAMPLE_M = 1 << SAMPLE_LOG2;   // samples per sampled tensor
 constexpr int SAMPLE_THREADS = 1024;
-constexpr int SAMPLE_PART = 2048;                          // samples per sampling block
-constexpr int SAMPLE_PART_PER_THREAD = SAMPLE_PART / SAMPLE_THREADS;
-constexpr int SAMPLE_PER_THREAD = SAMPLE_M / SAMPLE_THREADS;  // keys per thread in the merge
+constexpr int SAMPLE_PER_THREAD = SAMPLE_M / SAMPLE_THREADS;  // keys each thread holds
 constexpr int SAMPLE_BINS = 4096;    // key >> 19
 constexpr int K1_THREADS = 256;
 constexpr int WT = 1024;             // elements per warp tile
 constexpr int WT_VECS = WT / 128;    // float4 of each input per lane per warp tile
-constexpr int WT_CAP = 16;           // candidates staged per warp tile
+constexpr int WT_CAP = 16;           // candidate offsets staged per warp tile
+constexpr uint32_t STREAM_PREFETCH = 3;   // warp tiles per warp pulled into L2 early
 constexpr int ZERO_THREADS = 1024;
 
 // Per-tensor metadata written by the setup kernel.
@@ -41,7 +40,8 @@ struct SegMeta {
     uint32_t k;
     uint32_t T0;        // prefilter threshold key (NO_KEY when k == 0)
     uint32_t shift;     // relative digit: R1 = (key - T0) >> shift
-    uint32_t pad[3];
+    uint32_t t_ns[3];   // sampling block: ns from its start to the loaded samples,
+                        // the first histogram level and the end (diagnostics)
 };
 static_assert(sizeof(SegMeta) == 48, "SegMeta layout");
 
@@ -61,75 +61,59 @@ struct SetupParams {
     int64_t off[TCAP + 1];
     int64_t out_base[TCAP];
     uint32_t k[TCAP];
-    uint32_t* sample_keys;  // [T][SAMPLE_M] sampled keys
-    uint32_t* sample_done;  // [T] sampling blocks finished, cleared before the launch
-    int32_t n_sample_blocks;
     uint32_t m[TCAP];       // samples (0: no sampling; n: every element)
     uint32_t r[TCAP];       // target rank among the samples
     uint32_t r_hi[TCAP];    // rank of an upper estimate of the k-th key
-    uint16_t sampled[TCAP]; // i-th sampled tensor
-    uint16_t part_first[TCAP + 1];  // its first sampling block (prefix over sampled tensors)
+    uint16_t sampled[TCAP]; // i-th sampled tensor (block i samples it)
 };
 
-// The first n_sample_blocks blocks sample acc for the prefilter threshold T0
-// of the sampled tensors: every element when the tensor has at most SAMPLE_M
-// of them (then T0 is the exact k-th key), otherwise SAMPLE_M samples in 256
-// evenly spread runs of 64 consecutive elements (the loads coalesce).  Each
-// block computes SAMPLE_PART keys into the workspace; the last block of a
-// tensor to finish (a counter cleared before the launch) reads all of them
-// back from L2 and takes T0 as the r-th largest, in three histogram levels
-// (12 + 12 + 7 bits).  The shift of the relative digits is chosen so that
-// 4,095 bins of 2^shift keys above T0 reach twice past an upper estimate of
-// the k-th key.  The remaining blocks clear the workspace state of this call
-// and write the metadata of the tensors that are not sampled.
+// Block i < n_sampled samples acc for the prefilter threshold T0 of the i-th
+// sampled tensor: every element when the tensor has at most SAMPLE_M of them,
+// otherwise SAMPLE_M samples in 128 evenly spread runs of 64 consecutive
+// elements (the loads coalesce).  The keys stay in registers; T0 is the lower
+// edge of the bin of the r-th largest in two histogram levels (key bits 30..19,
+// then 18..7), so T0 <= that key.  The shift of the relative digits is
+// chosen so that 4,095 bins of 2^shift keys above T0 reach twice past an
+// upper estimate of the k-th key.  The remaining blocks clear the workspace
+// state of this call and write the metadata of the tensors not sampled.
 template <int TCAP>
 __global__ void __launch_bounds__(SAMPLE_THREADS)
 setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
     __shared__ uint32_t hist[SAMPLE_BINS];
     __shared__ uint32_t s_red[33];
     __shared__ FindResult s_fr;
-    __shared__ int s_last;
     const int b = blockIdx.x;
     const int tid = threadIdx.x;
-    if (b < p.n_sample_blocks) {
-        // which sampled tensor, which part of its samples
-        int i = 0, hi_i = p.n_sampled;
-        while (hi_i - i > 1) {
-            const int mid = (i + hi_i) >> 1;
-            if (p.part_first[mid] <= b) i = mid; else hi_i = mid;
-        }
-        const int l = p.sampled[i];
-        const int part = b - p.part_first[i];
-        const int parts = p.part_first[i + 1] - p.part_first[i];
+    // the streaming kernel may be scheduled now (it waits for this grid);
+    // this grid waits for the kernel before it on the stream
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (b < p.n_sampled) {
+        const int l = p.sampled[b];
         const int64_t off = p.off[l];
         const int64_t n = p.off[l + 1] - off;
         const uint32_t m = p.m[l];
         const bool full = (int64_t)m == n;
-        uint32_t* keys = p.sample_keys + (size_t)l * SAMPLE_M;
-#pragma unroll
-        for (int u = 0; u < SAMPLE_PART_PER_THREAD; ++u) {
-            const uint32_t s = (uint32_t)(part * SAMPLE_PART + u * SAMPLE_THREADS + tid);
-            if (s < m) {
-                // every element, or 256 runs of 64 consecutive elements
-                const int64_t pos = full ? off + s : off + (((int64_t)(s >> 6) * n) >> 8) + (s & 63);
-                keys[s] = key_of(__fmaf_rn(p.lr, __ldg(p.grad + pos), __ldg(p.resid + pos)));
-            }
-        }
-        // the last sampling block of the tensor computes the quantile
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) s_last = atomicAdd(&p.sample_done[l], 1u) == (uint32_t)(parts - 1);
-        __syncthreads();
-        if (!s_last) return;
-        __threadfence();
+        const uint64_t t_start = global_ns();
         for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
-        __syncthreads();
+        // every element, or 128 runs of 64 consecutive elements; all loads
+        // are issued before the first is used
+        float gv[SAMPLE_PER_THREAD], rv[SAMPLE_PER_THREAD];
+#pragma unroll
+        for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
+            const uint32_t s = (uint32_t)(u * SAMPLE_THREADS + tid);
+            const int64_t pos = full ? off + s : off + (((int64_t)(s >> 6) * n) >> 7) + (s & 63);
+            gv[u] = s < m ? __ldg(p.grad + pos) : 0.f;
+            rv[u] = s < m ? __ldg(p.resid + pos) : 0.f;
+        }
         uint32_t key[SAMPLE_PER_THREAD];
 #pragma unroll
         for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
             const uint32_t s = (uint32_t)(u * SAMPLE_THREADS + tid);
-            key[u] = s < m ? __ldcg(keys + s) : NO_KEY;
+            key[u] = s < m ? key_of(__fmaf_rn(p.lr, gv[u], rv[u])) : NO_KEY;
         }
+        __syncthreads();
+        const uint64_t t_loaded = global_ns();
         // level 1: key >> 19
 #pragma unroll
         for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
@@ -137,10 +121,11 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
         __syncthreads();
         block_find_bin(hist, SAMPLE_BINS, p.r[l], s_red, &s_fr);
         const uint32_t ok1 = s_fr.ok, b1 = s_fr.bin;
-        uint32_t rem = p.r[l] - s_fr.above;
+        const uint32_t rem = p.r[l] - s_fr.above;
         __syncthreads();
         block_find_bin(hist, SAMPLE_BINS, p.r_hi[l], s_red, &s_fr);
         const uint32_t bhi = s_fr.ok ? s_fr.bin : b1;
+        const uint64_t t_level1 = global_ns();
         // level 2: bits 18..7 of the keys in bin b1
         __syncthreads();
         for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
@@ -151,21 +136,9 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
         __syncthreads();
         block_find_bin(hist, SAMPLE_BINS, rem, s_red, &s_fr);
         const uint32_t ok2 = s_fr.ok, b2 = s_fr.bin;
-        rem -= s_fr.above;
-        // level 3: bits 6..0 of the keys in that sub-bin
-        __syncthreads();
-        for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
-        __syncthreads();
-        const uint32_t pre = (b1 << 12) | b2;
-#pragma unroll
-        for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
-            if (key[u] != NO_KEY && (key[u] >> 7) == pre) atomicAdd(&hist[key[u] & 127u], 1u);
-        __syncthreads();
-        block_find_bin(hist, SAMPLE_BINS, rem, s_red, &s_fr);
-        const uint32_t ok3 = s_fr.ok, b3 = s_fr.bin;
         if (tid == 0) {
             uint32_t T0 = 0;
-            if (ok1 && ok2 && ok3) T0 = (pre << 7) | b3;
+            if (ok1 && ok2) T0 = (b1 << 19) | (b2 << 7);
             // never above 0x7F800001: then "raw |x| bits >= T0" and "key >= T0"
             // agree for NaN too (lowering T0 only adds candidates)
             T0 = min(T0, 0x7F800001u);
@@ -181,12 +154,16 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
             sm.k = p.k[l];
             sm.T0 = T0;
             sm.shift = sh;
+            const uint64_t t_end = global_ns();
+            sm.t_ns[0] = (uint32_t)(t_loaded - t_start);
+            sm.t_ns[1] = (uint32_t)(t_level1 - t_start);
+            sm.t_ns[2] = (uint32_t)(t_end - t_start);
             p.meta[l] = sm;
         }
         return;
     }
-    const int zb = b - p.n_sample_blocks;
-    const int nz = gridDim.x - p.n_sample_blocks;
+    const int zb = b - p.n_sampled;
+    const int nz = gridDim.x - p.n_sampled;
     if (zb == 0) {
         if (tid == 0) {
             Ctrl c;
@@ -224,10 +201,7 @@ struct StreamParams {
     const SegMeta* meta;
     Ctrl* ctrl;
     uint32_t* wt_count;     // [num_wt] candidates of each warp tile (exact)
-    uint32_t* st_idx;       // [num_wt][WT_CAP] staged candidates, index order
-    float* st_val;
-    uint32_t* hist;         // [T][CHIST_WORDS]: candidate R1 at CH_R1, digit 1 at CH_C1
-    uint32_t* bound_before; // [T]: candidates of the warp tile holding off[l] below off[l]
+    uint16_t* wt_off;       // [num_wt][WT_CAP]: their offsets in the tile, unordered
 };
 
 // Tensor l with off[l] <= e < off[l+1] (empty tensors are skipped).
@@ -253,9 +227,6 @@ __device__ __forceinline__ int lower_bound_off(const int64_t* off, int T, int64_
 struct StreamShared {
     int64_t off[TCAP_LARGE + 1];
     uint32_t T0[TCAP_LARGE];
-    uint32_t sh[TCAP_LARGE];
-    uint32_t r1[REL_BINS];     // one tensor: candidate histograms in shared memory
-    uint32_t c1[D1_BINS];
 };
 
 // General warp tile: a partial last tile, a tile that spans tensors, or
@@ -296,93 +267,73 @@ __device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, cons
     return flags;
 }
 
-// Rare path of a warp tile with candidates: count them, stage them in index
-// order, add them to the candidate histograms (acc is read back from the
-// residual the warp has just written), and record the warp tile's count.
-__device__ __noinline__ void stream_tile_candidates(const StreamParams& p, StreamShared& S,
-                                                    uint32_t w, int64_t base, int l_lo, int l_hi,
-                                                    uint32_t flags, bool flat) {
+// Record the candidates of a warp tile: the exact count and, up to WT_CAP of
+// them, their offsets in the tile (lane-major, so not in index order; the
+// select kernel sorts each tile's few offsets and reads the values back from
+// the residual, which now holds acc).  Bit 4j + v of a lane's flags is offset
+// 128 j + 4 lane + v.
+__device__ __forceinline__ void stream_tile_stage(const StreamParams& p, uint32_t w, uint32_t flags) {
     const uint32_t lane = lane_id();
-    const uint32_t cnt = warp_sum((uint32_t)__popc(flags));
-    if (lane == 0) p.wt_count[w] = cnt;
-    uint32_t before = 0;   // candidates of earlier vectors
-    for (int j = 0; j < WT_VECS; ++j) {
-        const uint32_t fj = (flags >> (4 * j)) & 0xFu;
-        if (!__any_sync(0xFFFFFFFFu, fj != 0)) continue;
-        const uint32_t c = __popc(fj);
-        const uint32_t incl = warp_incl_scan(c);
-        uint32_t pos = before + incl - c;
-        const int64_t e = base + j * 128 + lane * 4;
-        for (int v = 0; v < 4; ++v) {
-            if (!((fj >> v) & 1u)) continue;
-            const float a = __ldcg(p.resid + e + v);
-            if (cnt <= WT_CAP) {
-                p.st_idx[(size_t)w * WT_CAP + pos] = (uint32_t)(e + v);
-                p.st_val[(size_t)w * WT_CAP + pos] = a;
-            }
-            const uint32_t key = key_of(a);
-            int l = l_lo;
-            while (l < l_hi && S.off[l + 1] <= e + v) ++l;
-            const uint32_t rb = min((key - S.T0[l]) >> S.sh[l], (uint32_t)(REL_BINS - 1));
-            if (flat) {
-                atomicAdd(&S.r1[rb], 1u);
-                atomicAdd(&S.c1[key >> 20], 1u);
-            } else {
-                atomicAdd(&p.hist[(size_t)l * CHIST_WORDS + CH_R1 + rb], 1u);
-                atomicAdd(&p.hist[(size_t)l * CHIST_WORDS + CH_C1 + (key >> 20)], 1u);
-            }
-            ++pos;
-        }
-        before += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    const uint32_t pc = (uint32_t)__popc(flags);
+    const uint32_t incl = warp_incl_scan(pc);
+    if (lane == 31) p.wt_count[w] = incl;
+    uint32_t pos = incl - pc;
+    uint16_t* dst = p.wt_off + (size_t)w * WT_CAP;
+    while (flags && pos < (uint32_t)WT_CAP) {
+        const uint32_t b = (uint32_t)(__ffs(flags) - 1);
+        flags &= flags - 1;
+        dst[pos++] = (uint16_t)(128u * (b >> 2) + 4u * lane + (b & 3u));
     }
 }
 
-// Tensors that start inside warp tile [base, tend): candidates below each start.
-__device__ __noinline__ void stream_tile_bounds(const StreamParams& p, const StreamShared& S,
-                                                int64_t base, int64_t tend, uint32_t flags) {
-    const uint32_t lane = lane_id();
-    const int T = p.T;
-    const int lb = max(1, lower_bound_off(S.off, T, base));
-    const int ub = min(T, lower_bound_off(S.off, T, tend));
-    for (int l = lb; l < ub; ++l) {
-        const int64_t bound = S.off[l];
-        uint32_t c = 0;
-        for (int j = 0; j < WT_VECS; ++j) {
-            const int64_t e = base + j * 128 + lane * 4;
-            for (int v = 0; v < 4; ++v) c += ((flags >> (j * 4 + v)) & 1u) && (e + v < bound);
-        }
-        c = warp_sum(c);
-        if (lane == 0) p.bound_before[l] = c;
-    }
+__device__ __forceinline__ void stream_tile_record(const StreamParams& p, uint32_t w,
+                                                   uint32_t flags) {
+    if (__any_sync(0xFFFFFFFFu, flags != 0)) stream_tile_stage(p, w, flags);
+    else if (lane_id() == 0) p.wt_count[w] = 0;
 }
 
 // The fused streaming pass, the only full sweep of the step:
 //   acc = fmaf(lr, grad, residual) written back to residual;
-//   candidates (key >= T0 of the element's tensor) staged per warp tile in
-//   index order (at most WT_CAP; the count is always exact);
-//   histograms of the candidates' relative digit 1 and digit 1 per tensor.
-// Each warp owns whole 1,024-element warp tiles (grid-stride), so warps never
-// wait for one another: the global order of the candidates is rebuilt by the
-// select kernel from the per-warp-tile counts.  The loop over full tiles of
-// one tensor is kept small; everything else is out of line.
+//   candidates (key >= T0 of the element's tensor) recorded per warp tile of
+//   1,024 elements: an exact count and the offsets of up to WT_CAP of them.
+// Each warp owns whole warp tiles, so warps never wait for one another; the
+// select kernel rebuilds the ordered candidate list from the records.  The loop
+// over full tiles of one tensor is kept small; everything else is out of line.
 template <bool VEC>
 __global__ void __launch_bounds__(K1_THREADS, 3)
-stream_kernel(const StreamParams p) {
+stream_kernel(const __grid_constant__ StreamParams p) {
     __shared__ StreamShared S;
     const int tid = threadIdx.x;
+    {
+        // While the setup kernel still runs (this grid is launched early),
+        // pull this warp's first warp tiles into L2: the reads do not depend
+        // on it, only the writes and the candidate test do.
+        const uint32_t warps = blockDim.x >> 5;
+        const uint32_t gw0 = blockIdx.x * warps + warp_id();
+        const uint32_t GW0 = gridDim.x * warps;
+        const uint32_t R0 = p.num_wt / GW0 >= 2 ? p.num_wt / GW0 - 1 : 0;
+        if (VEC && lane_id() == 0) {
+            for (uint32_t i = 0; i < STREAM_PREFETCH && i < R0; ++i) {
+                const int64_t base = (int64_t)(gw0 + i * GW0) * WT;
+                if (base + WT > p.N) break;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.grad + base),
+                             "r"((uint32_t)(WT * 4))
+                             : "memory");
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.resid + base),
+                             "r"((uint32_t)(WT * 4))
+                             : "memory");
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // setup_kernel's results
     const uint32_t lane = lane_id();
     const int T = p.T;
     const bool flat = (T == 1);
     for (int l = tid; l < T; l += blockDim.x) {
         S.off[l] = p.meta[l].off;
         S.T0[l] = p.meta[l].T0;
-        S.sh[l] = p.meta[l].shift;
     }
     if (tid == 0) S.off[T] = p.N;
-    if (flat) {
-        for (int i = tid; i < REL_BINS; i += blockDim.x) S.r1[i] = 0;
-        for (int i = tid; i < D1_BINS; i += blockDim.x) S.c1[i] = 0;
-    }
     __syncthreads();
 
     // Warp tiles are handed out statically for all but the last rounds, then
@@ -409,7 +360,6 @@ stream_kernel(const StreamParams p) {
         const int64_t tend = min(base + (int64_t)WT, p.N);
         const int l_lo = flat ? 0 : seg_of(S.off, T, base);
         const int l_hi = flat ? 0 : seg_of(S.off, T, tend - 1);
-        uint32_t flags = 0;
         if (VEC && l_lo == l_hi && tend - base == WT) {
             // full warp tile inside one tensor: 128-bit loads, no bounds checks
             const uint32_t T0 = S.T0[l_lo];
@@ -421,6 +371,7 @@ stream_kernel(const StreamParams p) {
                 gv[j] = ld_stream(g4 + 32 * j);
                 rv[j] = ld_stream(r4 + 32 * j);
             }
+            uint32_t flags = 0;
 #pragma unroll
             for (int j = 0; j < WT_VECS; ++j) {
                 float4 a;
@@ -434,23 +385,11 @@ stream_kernel(const StreamParams p) {
                 flags |= (uint32_t)((__float_as_uint(a.z) & KEY_MASK) >= T0) << (4 * j + 2);
                 flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0) << (4 * j + 3);
             }
+            stream_tile_record(p, w, flags);
         } else {
-            flags = stream_tile_general<VEC>(p, S, base, l_lo, l_hi);
+            stream_tile_record(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi));
         }
-        if (__any_sync(0xFFFFFFFFu, flags != 0)) {
-            stream_tile_candidates(p, S, w, base, l_lo, l_hi, flags, flat);
-        } else if (lane == 0) {
-            p.wt_count[w] = 0;
-        }
-        if (!flat) stream_tile_bounds(p, S, base, tend, flags);
         w = stat_next ? w + GW : R * GW + __shfl_sync(0xFFFFFFFFu, ticket, 0);
-    }
-    if (flat) {
-        __syncthreads();
-        for (int i = tid; i < REL_BINS; i += blockDim.x)
-            if (S.r1[i]) atomicAdd(&p.hist[CH_R1 + i], S.r1[i]);
-        for (int i = tid; i < D1_BINS; i += blockDim.x)
-            if (S.c1[i]) atomicAdd(&p.hist[CH_C1 + i], S.c1[i]);
     }
 }
 

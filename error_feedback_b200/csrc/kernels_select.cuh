@@ -11,10 +11,13 @@
 // magnitudes makes the set unique.)
 //
 // T is found by radix digits of the 31-bit key.  Standard digits are 11 + 10
-// + 10 bits; a prefiltered tensor of the compress step instead uses two
-// digits of key - T0 (see common.cuh), whose first histogram the streaming
-// pass already built and whose second is built while the candidates are
-// gathered, so that path needs no digit pass of its own.
+// + 10 bits (merge rounds, and the compress step's rescan of the residual).
+// A prefiltered tensor of the compress step instead uses two digits of
+// key - T0 (see common.cuh): the gather phase builds the first histogram
+// while it copies the candidates into one list in index order; the few
+// candidates in the k-th key's first-digit bin then go to a small per-tensor
+// entry list from which every block reads T, the tie quota and its own
+// output offset, so the candidate path needs three grid barriers in all.
 //
 // The grid is cooperative (all blocks resident): each block owns one
 // contiguous range of positions, histograms are summed in global memory and
@@ -34,6 +37,9 @@ constexpr int SEL_THREADS = 512;
 constexpr int SEG_MAX = 256;
 constexpr int EMIT_PER_THREAD = 4;
 constexpr int EMIT_TILE = SEL_THREADS * EMIT_PER_THREAD;
+// Entry list of a prefiltered tensor: candidates in the bin of relative digit
+// 1 that holds the k-th key, as (block << 12) | relative digit 2.
+constexpr uint32_t ENT_PER = 4096;
 
 struct Slot {
     int32_t l_first, l_last;
@@ -49,6 +55,14 @@ struct DigitState {
     uint32_t ok;       // 0: the counts did not add up (or relative overflow)
 };
 
+// Relative digit 1 of a prefiltered tensor, resolved.
+struct RelState {
+    uint32_t b1;    // bin of the k-th key
+    uint32_t rem;   // rank of the k-th key inside the bin
+    uint32_t cnt;   // candidates in the bin
+    uint32_t ok;    // 0: k == 0, or the counts did not add up
+};
+
 struct SelShared {
     int64_t seg[SEG_MAX + 1];
     __align__(16) uint32_t stage[REL_BINS];
@@ -57,13 +71,14 @@ struct SelShared {
     uint32_t red[33];
     uint32_t T0[SEG_MAX];
     uint32_t shift[SEG_MAX];
-    uint32_t b1[SEG_MAX];      // relative digit 1 of the k-th key (gather phase)
-    uint32_t a1[SEG_MAX];      // and the candidates above its bin
     FindResult fr;
+    RelState rs[2];            // first and last segment of the block's range
     DigitState ds;
     DigitState fin[2];         // final thresholds of the first and last segment
     int flag;
     uint32_t pre[4];
+    uint64_t ovf_pos[SEL_THREADS];   // gather: output position of each overflow tile
+    uint64_t before;                 // gather: output offset of the block
 };
 
 // Block-wide copy of n words (n a multiple of 4, 16-byte aligned) into
@@ -116,54 +131,33 @@ __device__ void resolve_std(const uint32_t* h1, const uint32_t* h2, const uint32
     __syncthreads();
 }
 
-// Relative digits of a prefiltered tensor.  With want_r2 false only digit 1
-// is resolved (S.ds.prefix = its bin); otherwise S.ds.prefix = T and
-// S.ds.rem = q.  ok = 0 when the k-th key lies above the covered range.
-__device__ void resolve_rel(const uint32_t* r1, const uint32_t* r2, uint32_t k, uint32_t T0,
-                            uint32_t shift, bool want_r2, SelShared& S,
-                            uint32_t known_b1 = 0xFFFFFFFFu, uint32_t known_a1 = 0) {
+// Relative digit 1 of a prefiltered tensor from its global histogram r1.
+__device__ RelState resolve_rel1(const uint32_t* r1, uint32_t k, SelShared& S) {
     __syncthreads();
-    if (k == 0) {
-        if (threadIdx.x == 0) S.ds = DigitState{1u, 0u, 0u, 1u};
-        __syncthreads();
-        return;
-    }
-    uint32_t ok, b1, rem;
-    if (known_b1 != 0xFFFFFFFFu) {
-        ok = 1;
-        b1 = known_b1;
-        rem = k - known_a1;
-    } else {
-        stage_words(S.stage, r1, REL_BINS, REL_BINS);
-        __syncthreads();
-        block_find_bin(S.stage, REL_BINS, k, S.red, &S.fr);
-        ok = (S.fr.ok && S.fr.bin != REL_BINS - 1) ? 1u : 0u;
-        b1 = S.fr.bin;
-        rem = k - S.fr.above;
-    }
-    uint32_t out = b1;
-    if (want_r2 && ok) {
-        __syncthreads();
-        const int nlow = 1 << shift;
-        if (nlow >= 4) {
-            stage_words(S.stage, r2, nlow, REL_BINS);
-        } else {
-            for (int i = threadIdx.x; i < REL_BINS; i += blockDim.x)
-                S.stage[i] = i < nlow ? r2[i] : 0u;
-        }
-        __syncthreads();
-        block_find_bin(S.stage, REL_BINS, rem, S.red, &S.fr);
-        ok = S.fr.ok;
-        rem -= S.fr.above;
-        out = T0 + (b1 << shift) + S.fr.bin;
-    }
-    if (threadIdx.x == 0) S.ds = DigitState{0u, out, rem, ok};
+    if (k == 0) return RelState{0u, 0u, 0u, 0u};
+    stage_words(S.stage, r1, REL_BINS, REL_BINS);
     __syncthreads();
+    block_find_bin(S.stage, REL_BINS, k, S.red, &S.fr);
+    const RelState r{S.fr.bin, k - S.fr.above, S.fr.cnt,
+                     (S.fr.ok && S.fr.bin != REL_BINS - 1) ? 1u : 0u};
+    __syncthreads();
+    return r;
+}
+
+// T (prefix) and the tie quota (rem) from the relative digit-2 histogram h2
+// (shared memory, REL_BINS words) of the k-th key's digit-1 bin.
+__device__ DigitState finish_rel(const uint32_t* h2, const RelState& rs, uint32_t T0,
+                                 uint32_t sh, SelShared& S) {
+    block_find_bin(h2, REL_BINS, rs.rem, S.red, &S.fr);
+    const DigitState d{0u, T0 + (rs.b1 << sh) + S.fr.bin, rs.rem - S.fr.above, S.fr.ok};
+    __syncthreads();
+    return d;
 }
 
 // ---------------------------------------------------------------- sources
 
-// Compress: candidates of the streaming pass, or the whole residual.
+// Compress: candidates of the streaming pass, or the whole residual.  The
+// generic digit passes below run only for the rescan of the residual.
 struct CompressSrc {
     float* resid;
     int64_t N;
@@ -178,9 +172,10 @@ struct CompressSrc {
     float* out_val;
     uint32_t num_wt;             // warp tiles of the streaming pass
     const uint32_t* wt_count;
-    const uint32_t* st_idx;      // [num_wt][WT_CAP]
-    const float* st_val;
-    const uint32_t* bound_before;
+    const uint16_t* wt_off;      // [num_wt][WT_CAP]
+    uint32_t* ent;               // [T][ENT_PER] entry lists
+    uint32_t* ent_cnt;           // [T] their lengths
+    uint64_t* agg;               // [grid] each block's candidate count + 1 (0: not yet)
     int32_t force_dense;
     int32_t dense;               // decided inside the kernel
 
@@ -188,13 +183,13 @@ struct CompressSrc {
     __device__ int64_t seg_bound(int l) const { return dense ? (l < T ? meta[l].off : N) : cand_start[l]; }
     __device__ uint32_t seg_k(int l) const { return meta[l].k; }
     __device__ uint32_t* h(int l, int part) const { return hist + (size_t)l * CHIST_WORDS + part; }
-    // whether segment l is resolved by standard digits
-    __device__ bool uses_std(int l) const {
-        if (dense) return true;
+    __device__ bool uses_std(int) const { return true; }
+    // the k-th key lies above the range of the relative digits
+    __device__ bool rel_overflow(int l) const {
         const uint32_t k = meta[l].k;
         return k > 0 && h(l, CH_R1)[REL_BINS - 1] >= k;
     }
-    __device__ uint32_t* d1(int l) const { return h(l, dense ? CH_D1 : CH_C1); }
+    __device__ uint32_t* d1(int l) const { return h(l, CH_D1); }
     __device__ uint32_t* d2(int l) const { return h(l, CH_D2); }
     __device__ uint32_t* d3(int l) const { return h(l, CH_D3); }
     __device__ void load(int64_t pos, uint32_t& idx, float& val) const {
@@ -208,13 +203,7 @@ struct CompressSrc {
         resid[idx] = 0.0f;
     }
     __device__ void resolve_final(int l, SelShared& S, uint32_t* status) const {
-        if (uses_std(l)) {
-            resolve_std(d1(l), d2(l), d3(l), seg_k(l), 3, S, status);
-        } else {
-            const SegMeta& m = meta[l];
-            resolve_rel(h(l, CH_R1), h(l, CH_R2), m.k, m.T0, m.shift, true, S, S.b1[l], S.a1[l]);
-            if (threadIdx.x == 0 && !S.ds.ok) atomicOr(status, ST_INCONSISTENT);
-        }
+        resolve_std(d1(l), d2(l), d3(l), seg_k(l), 3, S, status);
     }
 };
 
@@ -325,32 +314,249 @@ __device__ __forceinline__ void mark_phase(Ctrl* ctrl, int i) {
     if (blockIdx.x == 0 && threadIdx.x == 0) ctrl->t_phase[i] = global_ns();
 }
 
-// Gather-time bookkeeping of the second relative digit: a candidate of
-// tensor l whose first relative digit is the k-th's bin counts in the
-// tensor's digit-2 histogram.
-__device__ __forceinline__ void rel2_add(const CompressSrc& src, const SelShared& S, int l,
-                                         float v) {
-    const uint32_t b1 = S.b1[l];
-    if (b1 == 0xFFFFFFFFu) return;                 // tensor resolved otherwise
-    const uint32_t rel = key_of(v) - S.T0[l];
-    const uint32_t sh = S.shift[l];
-    if ((rel >> sh) == b1) atomicAdd(src.h(l, CH_R2) + (rel & ((1u << sh) - 1u)), 1u);
+// Output offset of a block inside segment l from the blocks before it: the
+// (gt, eq) counts of the run of earlier blocks whose ranges continue l (their
+// slots), summed by warp 0.  Result in S.pre[0..1].
+__device__ void chain_prefix(const SelCommon& cm, int c, int l, SelShared& S) {
+    if (threadIdx.x < 32) {
+        uint32_t pg = 0, pe = 0;
+        int cc = c - 1;
+        for (;;) {
+            const int j = cc - (int)lane_id();
+            bool match = false, cont = false;
+            uint32_t g = 0, e = 0;
+            if (j >= 0) {
+                const Slot sl = cm.slots[j];
+                match = sl.l_last == l;
+                cont = match && sl.l_first == l;
+                g = sl.gt_last;
+                e = sl.eq_last;
+            }
+            const uint32_t contm = __ballot_sync(0xFFFFFFFFu, cont);
+            const uint32_t matchm = __ballot_sync(0xFFFFFFFFu, match);
+            const uint32_t run = (contm == 0xFFFFFFFFu) ? 32u : (uint32_t)(__ffs(~contm) - 1);
+            const bool take = lane_id() < run || (lane_id() == run && ((matchm >> run) & 1u));
+            pg += warp_sum(take ? g : 0u);
+            pe += warp_sum(take ? e : 0u);
+            if (run < 32) break;
+            cc -= 32;
+        }
+        if (threadIdx.x == 0) {
+            S.pre[0] = pg;
+            S.pre[1] = pe;
+        }
+    }
+    __syncthreads();
 }
 
-// Gather phase of the compress select: rebuild the global candidate order
-// from the streaming pass's per-warp-tile staging.  Each block takes a
-// contiguous chunk of warp tiles; a grid barrier turns the chunk sums into
-// offsets; every staged candidate is copied to its place in the dense list,
-// and a warp tile that had more than WT_CAP candidates is rescanned from the
-// residual (which holds acc) with the same predicate.  Also records where
-// each tensor's candidates start, and builds the second relative digit of
-// the tensors that use it.  Then decides the path for every block alike:
-// candidates only if each tensor kept at least k of them and the list fit.
-// Returns false if a barrier gave up.
+// Ordered emission of positions [a, b) of segment l: key > Tk always, key ==
+// Tk while the tie quota q lasts; run_gt / run_eq are the counts of both
+// classes at positions of l before a.
+template <class Src>
+__device__ void emit_range(const Src& src, int l, int64_t a, int64_t b, uint32_t Tk, uint32_t q,
+                           uint32_t kseg, uint32_t run_gt, uint32_t run_eq, SelShared& S) {
+    const int tid = threadIdx.x;
+    for (int64_t base = a; base < b; base += EMIT_TILE) {
+        uint32_t idx[EMIT_PER_THREAD];
+        float val[EMIT_PER_THREAD];
+        uint32_t cls = 0;   // bit u: gt, bit 4+u: eq
+#pragma unroll
+        for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+            const int64_t pos = base + (int64_t)tid * EMIT_PER_THREAD + u;
+            idx[u] = DEAD;
+            val[u] = 0.f;
+            if (pos < b) src.load(pos, idx[u], val[u]);
+            if (idx[u] != DEAD) {
+                const uint32_t key = key_of(val[u]);
+                if (key > Tk) cls |= 1u << u;
+                else if (key == Tk) cls |= 1u << (4 + u);
+            }
+        }
+        const uint64_t mine = ((uint64_t)__popc(cls & 0xFu) << 32) | (uint64_t)__popc(cls >> 4);
+        uint64_t tot;
+        const uint64_t ex = block_excl_scan(mine, S.scan, &tot);
+        uint32_t g = run_gt + (uint32_t)(ex >> 32);
+        uint32_t e = run_eq + (uint32_t)(ex & 0xFFFFFFFFu);
+#pragma unroll
+        for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+            if ((cls >> u) & 1u) {
+                const uint32_t rank = g + (e < q ? e : q);
+                if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
+                ++g;
+            } else if ((cls >> (4 + u)) & 1u) {
+                if (e < q) {
+                    const uint32_t rank = g + e;
+                    if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
+                }
+                ++e;
+            }
+        }
+        run_gt += (uint32_t)(tot >> 32);
+        run_eq += (uint32_t)(tot & 0xFFFFFFFFu);
+    }
+}
+
+// ------------------------------------------------ compress candidate path
+
+// Relative digit-1 bin of a candidate of tensor l (key >= T0 of l).
+__device__ __forceinline__ uint32_t rel_bin(uint32_t key, uint32_t T0, uint32_t sh) {
+    return min((key - T0) >> sh, (uint32_t)(REL_BINS - 1));
+}
+
+__device__ __forceinline__ void r1_add(const CompressSrc& src, const SelShared& S, int l,
+                                       float v, uint32_t* s_r1) {
+    const uint32_t bin = rel_bin(key_of(v), S.T0[l], S.shift[l]);
+    if (s_r1) atomicAdd(&s_r1[bin], 1u);
+    else atomicAdd(src.h(l, CH_R1) + bin, 1u);
+}
+
+// Staged candidates of one warp tile, held by one thread: offsets (distinct,
+// slots >= cnt hold 0xFFFF, above every offset) and the values read back
+// from the residual (which holds acc).
+struct TileCands {
+    uint32_t o[WT_CAP];
+    float v[WT_CAP];
+};
+
+__device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, uint32_t cnt,
+                                            TileCands& t) {
+    const uint4* p4 = reinterpret_cast<const uint4*>(src.wt_off + (size_t)w * WT_CAP);
+    const uint4 a = p4[0];
+    t.o[0] = a.x & 0xFFFFu; t.o[1] = a.x >> 16; t.o[2] = a.y & 0xFFFFu; t.o[3] = a.y >> 16;
+    t.o[4] = a.z & 0xFFFFu; t.o[5] = a.z >> 16; t.o[6] = a.w & 0xFFFFu; t.o[7] = a.w >> 16;
+    uint4 b = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+    if (cnt > 8) b = p4[1];
+    t.o[8] = b.x & 0xFFFFu; t.o[9] = b.x >> 16; t.o[10] = b.y & 0xFFFFu; t.o[11] = b.y >> 16;
+    t.o[12] = b.z & 0xFFFFu; t.o[13] = b.z >> 16; t.o[14] = b.w & 0xFFFFu; t.o[15] = b.w >> 16;
+    const int64_t base = (int64_t)w * WT;
+#pragma unroll
+    for (int i = 0; i < WT_CAP; ++i) {
+        if ((uint32_t)i >= cnt) t.o[i] = 0xFFFFu;
+        t.v[i] = (uint32_t)i < cnt ? src.resid[base + t.o[i]] : 0.f;
+    }
+}
+
+// Write the staged candidates of warp tile w in index order (ranked by
+// offset) from position pos of the dense list, and add each to the relative
+// digit-1 histogram of its tensor: s_r1 (shared) when the caller's chunk
+// lies in tensor lc, else the global one.  S.seg holds element offsets.
+template <int C>
+__device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelShared& S,
+                                             uint32_t w, uint64_t pos, uint32_t cnt,
+                                             const TileCands& t, uint32_t* s_r1, int lc) {
+    const int64_t base = (int64_t)w * WT;
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+        if ((uint32_t)i >= cnt) continue;
+        uint32_t rank = 0;
+#pragma unroll
+        for (int j = 0; j < C; ++j) rank += t.o[j] < t.o[i];
+        const int64_t e = base + t.o[i];
+        const uint64_t q = pos + rank;
+        if (q < src.cap) {
+            src.cand_idx[q] = (uint32_t)e;
+            src.cand_val[q] = t.v[i];
+        }
+        r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), t.v[i], s_r1);
+    }
+}
+
+// Output offset of block c's candidates: the sum of the counts the blocks
+// before it published (count + 1; 0 = not yet), read by warp 0.  Every block
+// publishes before any heavy work and all blocks are resident, so the wait
+// is short; it is bounded all the same.
+__device__ uint64_t look_back(const uint64_t* agg, int c, uint32_t* status, SelShared& S) {
+    if (threadIdx.x < 32) {
+        uint64_t sum = 0;
+        for (int j = (int)lane_id(); j < c; j += 32) {
+            uint64_t v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
+            uint32_t it = 0;
+            while (v == 0) {
+                if (++it > SPIN_LIMIT) {
+                    atomicOr(status, ST_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);
+                v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
+            }
+            sum += v ? v - 1 : 0;
+        }
+        sum = warp_sum(sum);
+        if (threadIdx.x == 0) S.before = sum;
+    }
+    __syncthreads();
+    return S.before;
+}
+
+// Gather a warp tile with more than WT_CAP candidates (one warp): rescan it
+// from the residual (which holds acc) with the streaming pass's test.
+__device__ void gather_rescan(const CompressSrc& src, const SelShared& S, uint32_t w,
+                              uint64_t pos, uint32_t* s_r1, int lc) {
+    constexpr int U = 8;
+    const uint32_t lane = lane_id();
+    const int T = src.T;
+    const int64_t base = (int64_t)w * WT;
+    const int64_t tend = min(base + (int64_t)WT, src.N);
+    for (int64_t e0 = base; e0 < tend; e0 += 32 * U) {
+        float v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t e = e0 + 32 * u + lane;
+            v[u] = e < tend ? src.resid[e] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t e = e0 + 32 * u + lane;
+            bool f = false;
+            int l = lc;
+            if (e < tend) {
+                if (!s_r1) l = seg_of(S.seg, T, e);
+                f = key_of(v[u]) >= S.T0[l];
+            }
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, f);
+            if (f) {
+                const uint64_t q = pos + __popc(m & ((1u << lane) - 1u));
+                if (q < src.cap) {
+                    src.cand_idx[q] = (uint32_t)e;
+                    src.cand_val[q] = v[u];
+                }
+                r1_add(src, S, l, v[u], s_r1);
+            }
+            pos += __popc(m);
+        }
+    }
+}
+
+// Candidates of warp tile w below element bound (one thread).
+__device__ uint32_t tile_count_below(const CompressSrc& src, const SelShared& S, uint32_t w,
+                                     uint32_t cnt, int64_t bound) {
+    const int64_t base = (int64_t)w * WT;
+    uint32_t c = 0;
+    if (cnt <= (uint32_t)WT_CAP) {
+        for (uint32_t i = 0; i < cnt; ++i)
+            c += base + (int64_t)src.wt_off[(size_t)w * WT_CAP + i] < bound;
+    } else {
+        for (int64_t e = base; e < bound; ++e)
+            c += key_of(src.resid[e]) >= S.T0[seg_of(S.seg, src.T, e)];
+    }
+    return c;
+}
+
+// Gather phase of the compress select.  Each block takes a contiguous chunk
+// of warp tiles, publishes its candidate count at once and finds its output
+// offset by looking back at the counts of the blocks before it (no grid
+// barrier).  It copies its candidates, in index order, to [my0, my1) of the
+// dense list (the staged ones from registers loaded before the look-back;
+// tiles with more than WT_CAP candidates are rescanned), builds the relative
+// digit-1 histograms and records where each tensor's candidates start.
+// After one grid barrier every block takes the same decision: candidates
+// only if the list fit and each tensor kept at least k of them with its
+// k-th key inside the range of the relative digits.  Returns false if a
+// barrier gave up.
 __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
-                                SelShared& S) {
+                                SelShared& S, uint64_t& my0, uint64_t& my1) {
     const int G = gridDim.x, c = blockIdx.x, tid = threadIdx.x;
-    const uint32_t lane = lane_id(), warp = warp_id(), nwarps = blockDim.x >> 5;
+    const uint32_t warp = warp_id(), nwarps = blockDim.x >> 5;
     const int T = src.T;
     uint32_t* status = &cm.ctrl->status;
     int64_t* s_off = S.seg;
@@ -358,126 +564,91 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
         s_off[l] = src.meta[l].off;
         S.T0[l] = src.meta[l].T0;
         S.shift[l] = src.meta[l].shift;
-        S.b1[l] = 0xFFFFFFFFu;
     }
     if (tid == 0) s_off[T] = src.N;
-    __syncthreads();
     const uint32_t W = src.num_wt;
     const uint32_t per = (W + G - 1) / G;
     const uint32_t w0 = min((uint32_t)c * per, W), w1 = min(w0 + per, W);
 
-    // relative digit 1 of the tensors of this chunk (the k-th key's bin)
-    if (w0 < w1) {
-        const int tl0 = seg_of(s_off, T, (int64_t)w0 * WT);
-        const int tl1 = seg_of(s_off, T, min((int64_t)w1 * WT, src.N) - 1);
-        for (int l = tl0; l <= tl1; ++l) {
-            const SegMeta& m = src.meta[l];
-            if (m.k == 0 || src.uses_std(l)) continue;
-            resolve_rel(src.h(l, CH_R1), nullptr, m.k, m.T0, m.shift, false, S);
-            if (tid == 0) {
-                S.b1[l] = S.ds.ok ? S.ds.prefix : 0xFFFFFFFFu;
-                S.a1[l] = S.ds.ok ? m.k - S.ds.rem : 0u;
-            }
-        }
-    }
-
     uint32_t mine = 0;
     for (uint32_t w = w0 + tid; w < w1; w += blockDim.x) mine += src.wt_count[w];
     mine = block_sum(mine, S.red);
-    if (tid == 0) cm.slots[c].gt_first = mine;
-    if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return false;
-    mark_phase(cm.ctrl, 1);
-
-    uint64_t before = 0, total = 0;
-    for (int i = tid; i < G; i += blockDim.x) {
-        const uint64_t v = cm.slots[i].gt_first;
-        total += v;
-        if (i < c) before += v;
+    if (tid == 0) {
+        __threadfence();
+        *reinterpret_cast<volatile uint64_t*>(src.agg + c) = (uint64_t)mine + 1;
     }
-    before = block_sum(before, S.scan);
-    total = block_sum(total, S.scan);
-    const bool fits = total <= src.cap;
-    if (c == 0)
-        for (int l = tid; l <= T; l += blockDim.x)
-            if (l == 0) src.cand_start[0] = 0;
-            else if (s_off[l] >= src.N) src.cand_start[l] = (int64_t)total;
 
-    // overflow list in the stage buffer: pairs (warp tile, offset)
-    uint32_t* s_ovf_w = S.stage;
-    uint64_t* s_ovf_o = reinterpret_cast<uint64_t*>(S.stage + SEL_THREADS);
-    uint32_t* s_ovf_n = S.stage + 3 * SEL_THREADS;
-    uint64_t run = before;
-    for (uint32_t pw = w0; pw < w1; pw += blockDim.x) {
+    // relative digit 1 in shared memory when the whole chunk is in one tensor
+    const int64_t e0 = (int64_t)w0 * WT, e1 = min((int64_t)w1 * WT, src.N);
+    const int lc = w0 < w1 ? seg_of(s_off, T, e0) : 0;
+    const bool one = w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
+    uint32_t* s_r1 = one ? S.stage : nullptr;
+    if (one)
+        for (int i = tid; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
+    // tiles with more than WT_CAP candidates of a piece: (tile, position)
+    uint32_t* s_ovf_w = S.h1;
+    uint64_t before = 0, run = 0;
+    bool have_before = false;
+    for (uint32_t pw = w0; pw < w1 || !have_before; pw += blockDim.x) {
         const uint32_t w = pw + tid;
         const uint32_t cnt = w < w1 ? src.wt_count[w] : 0u;
-        if (tid == 0) *s_ovf_n = 0;
+        if (tid == 0) S.flag = 0;
         uint32_t piece;
         const uint32_t ex = block_excl_scan(cnt, S.red, &piece);
-        const uint64_t off = run + ex;
-        if (w < w1) {
+        TileCands tc;
+        const bool staged = cnt > 0 && cnt <= (uint32_t)WT_CAP;
+        if (staged) load_staged(src, w, cnt, tc);
+        if (!have_before) {
+            before = look_back(src.agg, c, status, S);
+            have_before = true;
+            mark_phase(cm.ctrl, 4);
+        }
+        const uint64_t pos = before + run + ex;
+        if (w < w1 && T > 1) {
             const int64_t base = (int64_t)w * WT;
             const int64_t tend = min(base + (int64_t)WT, src.N);
-            if (T > 1)
-                for (int l = max(1, lower_bound_off(s_off, T, base)); l < T && s_off[l] < tend; ++l)
-                    src.cand_start[l] = (int64_t)(off + src.bound_before[l]);
-            if (fits && cnt) {
-                if (cnt <= WT_CAP) {
-                    int l = seg_of(s_off, T, base);
-                    for (uint32_t i = 0; i < cnt; ++i) {
-                        const uint32_t idx = src.st_idx[(size_t)w * WT_CAP + i];
-                        const float v = src.st_val[(size_t)w * WT_CAP + i];
-                        src.cand_idx[off + i] = idx;
-                        src.cand_val[off + i] = v;
-                        while (l < T - 1 && s_off[l + 1] <= (int64_t)idx) ++l;
-                        rel2_add(src, S, l, v);
-                    }
-                } else {
-                    const uint32_t slot = atomicAdd(s_ovf_n, 1u);
-                    s_ovf_w[slot] = w;
-                    s_ovf_o[slot] = off;
-                }
-            }
+            for (int l = max(1, lower_bound_off(s_off, T, base)); l < T && s_off[l] < tend; ++l)
+                src.cand_start[l] = (int64_t)(pos + tile_count_below(src, S, w, cnt, s_off[l]));
+        }
+        if (cnt > (uint32_t)WT_CAP) {
+            const uint32_t slot = atomicAdd(reinterpret_cast<uint32_t*>(&S.flag), 1u);
+            s_ovf_w[slot] = w;
+            S.ovf_pos[slot] = pos;
+        } else if (cnt > 4) {
+            store_ranked<WT_CAP>(src, S, w, pos, cnt, tc, s_r1, lc);
+        } else if (cnt > 0) {
+            store_ranked<4>(src, S, w, pos, cnt, tc, s_r1, lc);
         }
         __syncthreads();
-        const uint32_t novf = *s_ovf_n;
-        for (uint32_t i = warp; i < novf; i += nwarps) {
-            const uint32_t w2 = s_ovf_w[i];
-            uint64_t pos = s_ovf_o[i];
-            const int64_t base = (int64_t)w2 * WT;
-            const int64_t tend = min(base + (int64_t)WT, src.N);
-            int l = seg_of(s_off, T, base);
-            for (int64_t e0 = base; e0 < tend; e0 += 32) {
-                const int64_t e = e0 + lane;
-                bool f = false;
-                float v = 0.f;
-                if (e < tend) {
-                    while (l < T - 1 && s_off[l + 1] <= e) ++l;
-                    v = src.resid[e];
-                    f = key_of(v) >= S.T0[l];
-                }
-                const uint32_t m = __ballot_sync(0xFFFFFFFFu, f);
-                if (f) {
-                    const uint64_t q = pos + __popc(m & ((1u << lane) - 1u));
-                    if (q < src.cap) {
-                        src.cand_idx[q] = (uint32_t)e;
-                        src.cand_val[q] = v;
-                    }
-                    rel2_add(src, S, l, v);
-                }
-                pos += __popc(m);
-                // keep the lanes' tensor cursors in step
-                l = __shfl_sync(0xFFFFFFFFu, l, 31);
-            }
-        }
+        const uint32_t novf = (uint32_t)S.flag;
+        for (uint32_t i = warp; i < novf; i += nwarps)
+            gather_rescan(src, S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
         __syncthreads();
         run += piece;
     }
+    my0 = before;
+    my1 = before + mine;
+    if (tid == 0) {
+        if (c == 0) src.cand_start[0] = 0;
+        if (c == G - 1)
+            for (int l = 1; l <= T; ++l)
+                if (s_off[l] >= src.N) src.cand_start[l] = (int64_t)my1;
+    }
+    if (one) {
+        uint32_t* g = src.h(lc, CH_R1);
+        for (int i = tid; i < REL_BINS; i += blockDim.x)
+            if (S.stage[i]) atomicAdd(&g[i], S.stage[i]);
+    }
+    mark_phase(cm.ctrl, 5);
     if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return false;
-    mark_phase(cm.ctrl, 2);
+    mark_phase(cm.ctrl, 1);
 
+    const uint64_t total = (uint64_t)src.cand_start[T];
+    const bool fits = total <= src.cap;
     uint32_t bad = 0;
     for (int l = tid; l < T; l += blockDim.x)
-        bad |= (uint64_t)(src.cand_start[l + 1] - src.cand_start[l]) < (uint64_t)src.meta[l].k;
+        bad |= ((uint64_t)(src.cand_start[l + 1] - src.cand_start[l]) < (uint64_t)src.meta[l].k) ||
+               src.rel_overflow(l);
     bad = block_sum(bad, S.red);
     src.dense = (src.force_dense || !fits || bad) ? 1 : 0;
     if (c == 0 && tid == 0) {
@@ -485,6 +656,224 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
         cm.ctrl->cand_total = total;
     }
     return true;
+}
+
+// One pass over positions [a, b) of prefiltered tensor l (block-wide) once
+// its digit-1 bin rs.b1 is known: returns the candidates above that bin, and
+// hands each candidate in the bin (its relative digit 2) to the entry list
+// of l (to_entries) or to the shared-memory histogram S.stage.
+__device__ uint32_t scan_rel_bin(const CompressSrc& src, int l, int64_t a, int64_t b,
+                                 const RelState& rs, bool to_entries, SelShared& S) {
+    const uint32_t T0 = S.T0[l], sh = S.shift[l];
+    const uint32_t lmask = (1u << sh) - 1u;
+    const uint32_t lane = lane_id();
+    uint32_t above = 0;
+    for (int64_t p0 = a; p0 < b; p0 += blockDim.x) {
+        const int64_t p = p0 + threadIdx.x;
+        bool hit = false;
+        uint32_t low = 0;
+        if (p < b) {
+            const uint32_t rel = key_of(src.cand_val[p]) - T0;
+            const uint32_t bin = min(rel >> sh, (uint32_t)(REL_BINS - 1));
+            above += bin > rs.b1;
+            hit = bin == rs.b1;
+            low = rel & lmask;
+        }
+        if (to_entries) {
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, hit);
+            if (m) {
+                const uint32_t lead = (uint32_t)(__ffs(m) - 1);
+                uint32_t at = 0;
+                if (lane == lead) at = atomicAdd(src.ent_cnt + l, (uint32_t)__popc(m));
+                at = __shfl_sync(0xFFFFFFFFu, at, lead);
+                if (hit)
+                    src.ent[(size_t)l * ENT_PER + at + __popc(m & ((1u << lane) - 1u))] =
+                        ((uint32_t)blockIdx.x << 12) | low;
+            }
+        } else if (hit) {
+            atomicAdd(&S.stage[low], 1u);
+        }
+    }
+    return block_sum(above, S.red);
+}
+
+__device__ __forceinline__ void zero_stage(SelShared& S) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
+    __syncthreads();
+}
+
+// Selection and emission on the dense candidate list.  The block's range
+// [a0, a1) is what it gathered.  A tensor that lies wholly inside the range
+// is finished here alone.  For the (at most two) tensors that cross the
+// range's ends: count the candidates above the k-th key's digit-1 bin (slot)
+// and put the candidates in the bin on the tensor's entry list; after a
+// barrier every block reads T, the tie quota and the entries of the blocks
+// before it from that list.  A bin with more than ENT_PER candidates uses a
+// global digit-2 histogram instead, and then all blocks exchange exact
+// (gt, eq) counts through one more barrier.
+__device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
+                                    SelShared& S, uint64_t a0, uint64_t a1) {
+    const int c = blockIdx.x, tid = threadIdx.x;
+    const int T = src.T;
+    uint32_t* status = &cm.ctrl->status;
+    __syncthreads();
+    for (int l = tid; l <= T; l += blockDim.x) S.seg[l] = src.cand_start[l];
+    __syncthreads();
+    const bool has = a1 > a0;
+    // an empty range passes the tensor running through it on to the next block
+    const int l_first = seg_of_pos(S.seg, T, (int64_t)a0);
+    const int l_last = has ? seg_of_pos(S.seg, T, (int64_t)a1 - 1) : l_first;
+    uint32_t A[2] = {0u, 0u};
+    bool cross[2] = {false, false};
+    for (int l = l_first; has && l <= l_last; ++l) {
+        const int64_t a = max((int64_t)a0, S.seg[l]);
+        const int64_t b = min((int64_t)a1, S.seg[l + 1]);
+        if (a >= b) continue;
+        const uint32_t k = src.meta[l].k;
+        const RelState rs = resolve_rel1(src.h(l, CH_R1), k, S);
+        if (!rs.ok) {
+            if (k && tid == 0) atomicOr(status, ST_INCONSISTENT);
+            continue;
+        }
+        const bool local = S.seg[l] >= (int64_t)a0 && S.seg[l + 1] <= (int64_t)a1;
+        if (local) {
+            zero_stage(S);
+            scan_rel_bin(src, l, a, b, rs, false, S);
+            __syncthreads();
+            const DigitState d = finish_rel(S.stage, rs, S.T0[l], S.shift[l], S);
+            if (!d.ok) {
+                if (tid == 0) atomicOr(status, ST_INCONSISTENT);
+                continue;
+            }
+            emit_range(src, l, a, b, d.prefix, d.rem, k, 0u, 0u, S);
+            continue;
+        }
+        const bool fast = rs.cnt <= ENT_PER;
+        if (!fast) zero_stage(S);
+        const uint32_t above = scan_rel_bin(src, l, a, b, rs, fast, S);
+        if (!fast) {
+            __syncthreads();
+            uint32_t* g = src.h(l, CH_R2);
+            for (int i = tid; i < REL_BINS; i += blockDim.x)
+                if (S.stage[i]) atomicAdd(&g[i], S.stage[i]);
+            if (tid == 0) atomicOr(&cm.ctrl->r2_path, 1u);
+        }
+        if (l == l_first) {
+            if (tid == 0) S.rs[0] = rs;
+            A[0] = above;
+            cross[0] = true;
+        } else {
+            if (tid == 0) S.rs[1] = rs;
+            A[1] = above;
+            cross[1] = true;
+        }
+    }
+    if (tid == 0) {
+        Slot sl;
+        sl.l_first = l_first;
+        sl.l_last = l_last;
+        sl.gt_first = A[0];
+        sl.eq_first = 0;
+        sl.gt_last = l_first == l_last ? A[0] : A[1];
+        sl.eq_last = 0;
+        sl.pad[0] = sl.pad[1] = 0;
+        cm.slots[c] = sl;
+    }
+    if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
+    mark_phase(cm.ctrl, 2);
+    const bool r2p = *reinterpret_cast<volatile uint32_t*>(&cm.ctrl->r2_path) != 0;
+
+    // T and the tie quota of the crossing tensors
+    DigitState fin[2];
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+        fin[side] = DigitState{1u, 0u, 0u, 0u};
+        if (!cross[side]) continue;
+        const int l = side == 0 ? l_first : l_last;
+        const RelState rs = S.rs[side];
+        zero_stage(S);
+        if (rs.cnt <= ENT_PER) {
+            const uint32_t E = min(*reinterpret_cast<volatile uint32_t*>(src.ent_cnt + l), ENT_PER);
+            const uint32_t* el = src.ent + (size_t)l * ENT_PER;
+            for (uint32_t i = tid; i < E; i += blockDim.x) atomicAdd(&S.stage[el[i] & 4095u], 1u);
+        } else {
+            stage_words(S.stage, src.h(l, CH_R2), REL_BINS, REL_BINS);
+        }
+        __syncthreads();
+        fin[side] = finish_rel(S.stage, rs, S.T0[l], S.shift[l], S);
+        if (!fin[side].ok && tid == 0) atomicOr(status, ST_INCONSISTENT);
+    }
+    if (r2p) {
+        // exact counts of both classes per block
+        uint32_t gt[2] = {0u, 0u}, eq[2] = {0u, 0u};
+#pragma unroll
+        for (int side = 0; side < 2; ++side) {
+            if (!cross[side] || !fin[side].ok) continue;
+            const int l = side == 0 ? l_first : l_last;
+            const int64_t a = max((int64_t)a0, S.seg[l]);
+            const int64_t b = min((int64_t)a1, S.seg[l + 1]);
+            const uint32_t Tk = fin[side].prefix;
+            uint32_t g = 0, e = 0;
+            for (int64_t p = a + tid; p < b; p += blockDim.x) {
+                const uint32_t key = key_of(src.cand_val[p]);
+                g += key > Tk;
+                e += key == Tk;
+            }
+            gt[side] = block_sum(g, S.red);
+            eq[side] = block_sum(e, S.red);
+        }
+        if (tid == 0) {
+            Slot sl;
+            sl.l_first = l_first;
+            sl.l_last = l_last;
+            sl.gt_first = gt[0];
+            sl.eq_first = eq[0];
+            sl.gt_last = l_first == l_last ? gt[0] : gt[1];
+            sl.eq_last = l_first == l_last ? eq[0] : eq[1];
+            sl.pad[0] = sl.pad[1] = 0;
+            cm.slots[c] = sl;
+        }
+        if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
+        mark_phase(cm.ctrl, 3);
+    }
+    mark_phase(cm.ctrl, 6);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+        if (!cross[side] || !fin[side].ok) continue;
+        if (side == 1 && l_last == l_first) continue;
+        const int l = side == 0 ? l_first : l_last;
+        const int64_t a = max((int64_t)a0, S.seg[l]);
+        const int64_t b = min((int64_t)a1, S.seg[l + 1]);
+        uint32_t pg = 0, pe = 0;
+        if (side == 0 && a > S.seg[l]) {
+            chain_prefix(cm, c, l, S);
+            pg = S.pre[0];
+            pe = S.pre[1];
+            __syncthreads();
+            if (!r2p) {
+                // candidates of the k-th key's bin held by earlier blocks
+                const RelState rs = S.rs[0];
+                const uint32_t t = fin[0].prefix - S.T0[l] - (rs.b1 << S.shift[l]);
+                const uint32_t E = min(src.ent_cnt[l], ENT_PER);
+                const uint32_t* el = src.ent + (size_t)l * ENT_PER;
+                uint32_t g = 0, e = 0;
+                for (uint32_t i = tid; i < E; i += blockDim.x) {
+                    const uint32_t v = el[i];
+                    if ((int)(v >> 12) < c) {
+                        g += (v & 4095u) > t;
+                        e += (v & 4095u) == t;
+                    }
+                }
+                pg += block_sum(g, S.red);
+                pe += block_sum(e, S.red);
+            }
+        }
+        emit_range(src, l, a, b, fin[side].prefix, fin[side].rem, src.meta[l].k, pg, pe, S);
+    }
+    mark_phase(cm.ctrl, 7);
 }
 
 // ---------------------------------------------------------------- kernel
@@ -502,14 +891,13 @@ select_kernel(Src src, SelCommon cm) {
 
     int first_digit;
     if constexpr (std::is_same<Src, CompressSrc>::value) {
-        if (!compress_gather(src, cm, epoch, S)) return;
-        // digit passes: all three on the rescan path; on the candidate path
-        // digits 2 and 3 only if some tensor uses standard digits
-        uint32_t need = 0;
-        if (!src.dense)
-            for (int l = tid; l < src.T; l += blockDim.x) need |= src.uses_std(l) ? 1u : 0u;
-        need = block_sum(need, S.red);
-        first_digit = src.dense ? 1 : (need ? 2 : 4);
+        uint64_t my0, my1;
+        if (!compress_gather(src, cm, epoch, S, my0, my1)) return;
+        if (!src.dense) {
+            compress_candidates(src, cm, epoch, S, my0, my1);
+            return;
+        }
+        first_digit = 1;
     } else {
         src.fold_bad_input(cm.ctrl);
         first_digit = src.d1_done ? 2 : 1;
@@ -609,6 +997,9 @@ select_kernel(Src src, SelCommon cm) {
     }
     if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
     mark_phase(cm.ctrl, 6);
+    // a kernel launched after this one with programmatic serialisation may be
+    // scheduled now; it still waits for this grid to finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- emission
     for (int l = l_first; l <= l_last; ++l) {
@@ -623,81 +1014,14 @@ select_kernel(Src src, SelCommon cm) {
             fs = S.ds;
         }
         if (fs.none || !fs.ok) continue;
-        const uint32_t Tk = fs.prefix;
-        const uint32_t q = fs.rem;
-        const uint32_t kseg = src.seg_k(l);
-        // counts of earlier blocks in this segment
-        if (tid < 32) {
-            uint32_t pg = 0, pe = 0;
-            if (l == l_first && a > S.seg[l]) {
-                int cc = c - 1;
-                for (;;) {
-                    const int j = cc - (int)lane_id();
-                    bool match = false, cont = false;
-                    uint32_t g = 0, e = 0;
-                    if (j >= 0) {
-                        const Slot sl = cm.slots[j];
-                        match = sl.l_last == l;
-                        cont = match && sl.l_first == l;
-                        g = sl.gt_last;
-                        e = sl.eq_last;
-                    }
-                    const uint32_t contm = __ballot_sync(0xFFFFFFFFu, cont);
-                    const uint32_t matchm = __ballot_sync(0xFFFFFFFFu, match);
-                    const uint32_t run = (contm == 0xFFFFFFFFu) ? 32u : (uint32_t)(__ffs(~contm) - 1);
-                    const bool take = lane_id() < run || (lane_id() == run && ((matchm >> run) & 1u));
-                    pg += warp_sum(take ? g : 0u);
-                    pe += warp_sum(take ? e : 0u);
-                    if (run < 32) break;
-                    cc -= 32;
-                }
-            }
-            if (tid == 0) {
-                S.pre[0] = pg;
-                S.pre[1] = pe;
-            }
+        uint32_t pg = 0, pe = 0;
+        if (l == l_first && a > S.seg[l]) {
+            chain_prefix(cm, c, l, S);
+            pg = S.pre[0];
+            pe = S.pre[1];
+            __syncthreads();
         }
-        __syncthreads();
-        uint32_t run_gt = S.pre[0], run_eq = S.pre[1];
-        __syncthreads();
-        for (int64_t base = a; base < b; base += EMIT_TILE) {
-            uint32_t idx[EMIT_PER_THREAD];
-            float val[EMIT_PER_THREAD];
-            uint32_t cls = 0;   // bit u: gt, bit 4+u: eq
-#pragma unroll
-            for (int u = 0; u < EMIT_PER_THREAD; ++u) {
-                const int64_t pos = base + (int64_t)tid * EMIT_PER_THREAD + u;
-                idx[u] = DEAD;
-                val[u] = 0.f;
-                if (pos < b) src.load(pos, idx[u], val[u]);
-                if (idx[u] != DEAD) {
-                    const uint32_t key = key_of(val[u]);
-                    if (key > Tk) cls |= 1u << u;
-                    else if (key == Tk) cls |= 1u << (4 + u);
-                }
-            }
-            const uint64_t mine = ((uint64_t)__popc(cls & 0xFu) << 32) | (uint64_t)__popc(cls >> 4);
-            uint64_t tot;
-            const uint64_t ex = block_excl_scan(mine, S.scan, &tot);
-            uint32_t g = run_gt + (uint32_t)(ex >> 32);
-            uint32_t e = run_eq + (uint32_t)(ex & 0xFFFFFFFFu);
-#pragma unroll
-            for (int u = 0; u < EMIT_PER_THREAD; ++u) {
-                if ((cls >> u) & 1u) {
-                    const uint32_t rank = g + (e < q ? e : q);
-                    if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
-                    ++g;
-                } else if ((cls >> (4 + u)) & 1u) {
-                    if (e < q) {
-                        const uint32_t rank = g + e;
-                        if (rank < kseg) src.emit(l, rank, idx[u], val[u]);
-                    }
-                    ++e;
-                }
-            }
-            run_gt += (uint32_t)(tot >> 32);
-            run_eq += (uint32_t)(tot & 0xFFFFFFFFu);
-        }
+        emit_range(src, l, a, b, fs.prefix, fs.rem, src.seg_k(l), pg, pe, S);
     }
     mark_phase(cm.ctrl, 7);
 }

@@ -14,6 +14,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "topk_ef.h"
@@ -42,8 +43,9 @@ int cuda_fail(cudaError_t e) {
 }
 
 // ------------------------------------------------------------------ tracing
-// When enabled, every kernel launch is bracketed by two CUDA events on the
-// call's stream; records accumulate until they are read back.
+// When enabled, every kernel launch (or only those of one kernel) is
+// bracketed by two CUDA events on the call's stream; records accumulate until
+// they are read back.
 
 constexpr int TRACE_MAX = 4096;
 
@@ -51,6 +53,10 @@ struct Trace {
     int on = 0;
     int dev = -1;
     int n = 0;
+    bool open = false;          // a launch is bracketed by its first event
+    std::string only;           // trace only this kernel (empty: all)
+    int every = 1;              // and of those only every every-th launch
+    uint64_t seen = 0;          // launches that passed the name filter
     cudaEvent_t ev[2 * TRACE_MAX] = {};
     const char* name[TRACE_MAX] = {};
 };
@@ -58,13 +64,18 @@ Trace g_trace;
 std::mutex g_trace_mu;
 
 void trace_before(cudaStream_t st, const char* name) {
+    g_trace.open = false;
     if (!g_trace.on || g_trace.n >= TRACE_MAX) return;
+    if (!g_trace.only.empty() && g_trace.only != name) return;
+    if (g_trace.seen++ % (uint64_t)g_trace.every != 0) return;
     g_trace.name[g_trace.n] = name;
     cudaEventRecord(g_trace.ev[2 * g_trace.n], st);
+    g_trace.open = true;
 }
 
 void trace_after(cudaStream_t st) {
-    if (!g_trace.on || g_trace.n >= TRACE_MAX) return;
+    if (!g_trace.open) return;
+    g_trace.open = false;
     cudaEventRecord(g_trace.ev[2 * g_trace.n + 1], st);
     ++g_trace.n;
 }
@@ -108,6 +119,24 @@ int device_facts(DevFacts* out) {
     }
     *out = g_facts[dev];
     return TOPK_EF_OK;
+}
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel on the stream is still running, and waits for it
+// (griddepcontrol.wait) before touching anything that kernel produces.
+template <typename Kern, typename Arg>
+cudaError_t launch_pdl(Kern kernel, int grid, int block, cudaStream_t st, const Arg& arg) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, arg);
 }
 
 // ------------------------------------------------------- compress planning
@@ -161,8 +190,8 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
 
 // Workspace layout of one compress group (<= TCAP_LARGE tensors).
 struct CLayout {
-    size_t ctrl, meta, sample_done, zero_begin, cand_start, hist, zero_end, bound_before, wt_count,
-        st_idx, st_val, sample_keys, slots, cand_idx, cand_val, total;
+    size_t ctrl, meta, zero_begin, cand_start, ent_cnt, agg, hist, zero_end, wt_count, wt_off,
+        ent, slots, cand_idx, cand_val, total;
     int64_t cap;
     uint32_t num_wt;
 };
@@ -179,24 +208,22 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + sizeof(Ctrl));
     L.meta = o;
     o = align_up(o + T * sizeof(SegMeta));
-    L.sample_done = o;
-    o = align_up(o + T * sizeof(uint32_t));
     L.zero_begin = o;
     L.cand_start = o;
     o = align_up(o + (T + 1) * sizeof(int64_t));
+    L.ent_cnt = o;
+    o = align_up(o + T * sizeof(uint32_t));
+    L.agg = o;
+    o = align_up(o + SLOT_MAX * sizeof(uint64_t));
     L.hist = o;
     o = align_up(o + T * CHIST_WORDS * sizeof(uint32_t));
     L.zero_end = o;
-    L.bound_before = o;
-    o = align_up(o + (T + 1) * sizeof(uint32_t));
     L.wt_count = o;
     o = align_up(o + (size_t)L.num_wt * sizeof(uint32_t));
-    L.st_idx = o;
-    o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(uint32_t));
-    L.st_val = o;
-    o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(float));
-    L.sample_keys = o;
-    o = align_up(o + T * (size_t)SAMPLE_M * sizeof(uint32_t));
+    L.wt_off = o;
+    o = align_up(o + (size_t)L.num_wt * WT_CAP * sizeof(uint16_t));
+    L.ent = o;
+    o = align_up(o + T * (size_t)ENT_PER * sizeof(uint32_t));
     L.slots = o;
     o = align_up(o + SLOT_MAX * sizeof(Slot));
     L.cand_idx = o;
@@ -263,9 +290,7 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
     p.meta = reinterpret_cast<SegMeta*>(ws + L.meta);
     p.zero_ptr = reinterpret_cast<uint4*>(ws + L.zero_begin);
     p.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
-    p.sample_keys = reinterpret_cast<uint32_t*>(ws + L.sample_keys);
-    p.sample_done = reinterpret_cast<uint32_t*>(ws + L.sample_done);
-    int ns = 0, blocks = 0;
+    int ns = 0;
     for (int l = 0; l < T; ++l) {
         const TensorPlan& t = g.plans[l];
         p.off[l] = t.off;
@@ -274,25 +299,13 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
         p.m[l] = force_t0_zero ? 0u : t.m;
         p.r[l] = t.r;
         p.r_hi[l] = t.r_hi;
-        if (p.m[l]) {
-            p.sampled[ns] = (uint16_t)l;
-            p.part_first[ns] = (uint16_t)blocks;
-            blocks += (int)((p.m[l] + SAMPLE_PART - 1) / SAMPLE_PART);
-            ++ns;
-        }
+        if (p.m[l]) p.sampled[ns++] = (uint16_t)l;
     }
-    p.part_first[ns] = (uint16_t)blocks;
     p.off[T] = g.N;
     p.n_sampled = ns;
-    p.n_sample_blocks = blocks;
-    if (blocks) {
-        cudaError_t e = cudaMemsetAsync(ws + L.sample_done, 0, T * sizeof(uint32_t), st);
-        if (e != cudaSuccess) return e;
-    }
     const uint64_t per_block = (uint64_t)ZERO_THREADS * 8;
     const int nz = (int)std::max<uint64_t>(1, std::min<uint64_t>(148, (p.zero_vec4 + per_block - 1) / per_block));
-    setup_kernel<TCAP><<<blocks + nz, SAMPLE_THREADS, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(setup_kernel<TCAP>, ns + nz, SAMPLE_THREADS, st, p);
 }
 
 int compress_group(const Group& g, const float* grad, float* resid, float lr, int32_t* out_idx,
@@ -323,17 +336,14 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     sp.meta = reinterpret_cast<const SegMeta*>(ws + L.meta);
     sp.ctrl = ctrl;
     sp.wt_count = reinterpret_cast<uint32_t*>(ws + L.wt_count);
-    sp.st_idx = reinterpret_cast<uint32_t*>(ws + L.st_idx);
-    sp.st_val = reinterpret_cast<float*>(ws + L.st_val);
-    sp.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
-    sp.bound_before = reinterpret_cast<uint32_t*>(ws + L.bound_before);
+    sp.wt_off = reinterpret_cast<uint16_t*>(ws + L.wt_off);
     const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
     const int64_t warps_needed = L.num_wt;
     const int g1 = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(warps_needed, K1_THREADS / 32),
                                                                (int64_t)f.sms * f.k1_blocks));
     trace_before(st, "stream_kernel");
-    if (vec) stream_kernel<true><<<g1, K1_THREADS, 0, st>>>(sp);
-    else stream_kernel<false><<<g1, K1_THREADS, 0, st>>>(sp);
+    e = vec ? launch_pdl(stream_kernel<true>, g1, K1_THREADS, st, sp)
+            : launch_pdl(stream_kernel<false>, g1, K1_THREADS, st, sp);
     trace_after(st);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
 
@@ -347,21 +357,24 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     src.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
     src.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
     src.cap = (uint64_t)L.cap;
-    src.hist = sp.hist;
+    src.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
     src.out_idx = out_idx;
     src.out_val = out_val;
     src.num_wt = L.num_wt;
     src.wt_count = sp.wt_count;
-    src.st_idx = sp.st_idx;
-    src.st_val = sp.st_val;
-    src.bound_before = sp.bound_before;
+    src.wt_off = sp.wt_off;
+    src.ent = reinterpret_cast<uint32_t*>(ws + L.ent);
+    src.ent_cnt = reinterpret_cast<uint32_t*>(ws + L.ent_cnt);
+    src.agg = reinterpret_cast<uint64_t*>(ws + L.agg);
     src.force_dense = force_dense ? 1 : 0;
     src.dense = 0;
     SelCommon cm;
     cm.ctrl = ctrl;
     cm.bar = &ctrl->bar;
     cm.slots = reinterpret_cast<Slot*>(ws + L.slots);
-    const int G = std::min(SLOT_MAX, f.sms * f.selc_blocks);
+    // one block per SM: cheaper grid barriers, no less bandwidth for the
+    // small candidate list (the rescan fallback is still memory bound)
+    const int G = std::min(SLOT_MAX, f.sms * std::min(1, f.selc_blocks));
     void* args[] = {&src, &cm};
     trace_before(st, "select_kernel<CompressSrc>");
     e = cudaLaunchCooperativeKernel((const void*)select_kernel<CompressSrc>, dim3(G),
@@ -629,8 +642,9 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
         ms.pair_stride = 1;
         cm.bar = &ctrl->merge_bar[0];
         void* args[] = {&ms, &cm};
+        const int G1 = (int)std::max<int64_t>(1, std::min<int64_t>(G, ceil_div64(k_in, 4096)));
         trace_before(st, "select_kernel<MergeSrc>");
-        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(G),
+        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(G1),
                                         dim3(SEL_THREADS), args, 0, st);
         trace_after(st);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -672,8 +686,11 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
         }
         cm.bar = &ctrl->merge_bar[r];
         void* args[] = {&ms, &cm};
+        // about 4,096 merged positions per block: small rounds use few blocks
+        const int Gr = (int)std::max<int64_t>(
+            1, std::min<int64_t>(G, ceil_div64((int64_t)L.np[r] * L.mcap[r], 4096)));
         trace_before(st, "select_kernel<MergeSrc>");
-        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(G),
+        e = cudaLaunchCooperativeKernel((const void*)select_kernel<MergeSrc>, dim3(Gr),
                                         dim3(SEL_THREADS), args, 0, st);
         trace_after(st);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -712,11 +729,17 @@ int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns) {
     if (!ws || !ns) return TOPK_EF_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     Ctrl c;
+    SegMeta m0;
     cudaError_t e = cudaMemcpyAsync(&c, ws, sizeof(c), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&m0, static_cast<const char*>(ws) + align_up(sizeof(Ctrl)), sizeof(m0),
+                            cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
     for (int i = 0; i < 8; ++i)
         ns[i] = c.t_phase[i] ? (int64_t)(c.t_phase[i] - c.t_phase[0]) : -1;
+    for (int i = 0; i < 3; ++i) ns[8 + i] = m0.t_ns[2] ? (int64_t)m0.t_ns[i] : -1;
+    ns[11] = -1;
     return TOPK_EF_OK;
 }
 
@@ -757,6 +780,16 @@ int topk_ef_trace_enable(int on) {
     }
     g_trace.on = on ? 1 : 0;
     g_trace.n = 0;
+    g_trace.open = false;
+    g_trace.seen = 0;
+    return TOPK_EF_OK;
+}
+
+int topk_ef_trace_only(const char* kernel_name, int every) {
+    if (every < 1) return TOPK_EF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    g_trace.only = kernel_name ? kernel_name : "";
+    g_trace.every = every;
     return TOPK_EF_OK;
 }
 

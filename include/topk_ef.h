@@ -202,11 +202,17 @@ const char* topk_ef_status_string(int status);
 int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
 
 /*
- * Diagnostics of the last call on `ws` (synchronises `stream`): for the
- * select kernel's block 0, the time in nanoseconds from the kernel's start to
- * the end of each phase: ns[1], ns[2] the two gather barriers (compress),
- * ns[3..5] digit passes 1..3, ns[6] the count barrier, ns[7] the end of the
- * emission; -1 for a phase that did not run.  `ns` is host memory of 8 int64.
+ * Diagnostics of the last compress call on `ws` (synchronises `stream`), in
+ * nanoseconds; -1 for a step that did not run.  `ns` is host memory of 12
+ * int64.  ns[0..7]: block 0 of the select kernel, from the kernel's start:
+ *   candidate path: ns[4] offset look-back done, ns[5] gather done,
+ *     ns[1] first grid barrier, ns[2] second grid barrier, ns[3] barrier of
+ *     the exact-count exchange (only when a bin overflowed its entry list),
+ *     ns[6] emission starts, ns[7] end;
+ *   rescan fallback: ns[1] gather barrier, ns[3..5] the barriers after
+ *     digit passes 1..3, ns[6] the count barrier, ns[7] end.
+ * ns[8..10]: the sampling block of the first tensor, from its start: samples
+ * loaded, first histogram level resolved, end.  ns[11] is reserved (-1).
  */
 int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns);
 
@@ -231,9 +237,16 @@ int topk_ef_set_test_flags(int flags);
  *       (host float[max]) and kernel name (host const char*[max], static
  *       strings) of the first min(max, recorded) of them, sets *count to that
  *       number and clears the record.
+ *   topk_ef_trace_only(name, every)    record only the launches of the
+ *       kernel with this name (as topk_ef_trace_read reports it, e.g.
+ *       "stream_kernel"), and of those the 1st, (every+1)-th, ... after
+ *       tracing was enabled, so that the other launches keep running back to
+ *       back; NULL or "" selects every kernel again.  The string is copied.
+ *       every < 1: TOPK_EF_ERR_INVALID_ARG.
  */
 int topk_ef_trace_enable(int on);
 int topk_ef_trace_read(float* ms, const char** names, int max_entries, int* count);
+int topk_ef_trace_only(const char* kernel_name, int every);
 
 #ifdef __cplusplus
 }

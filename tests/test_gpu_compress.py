@@ -105,13 +105,14 @@ def test_forced_fallback(flags):
 
 
 def test_sampler_defeated():
-    """Only the strided sample positions hold large values, so the threshold
-    estimate sits above the k-th magnitude (fewer than k candidates): the
-    rescan fallback must give the exact answer."""
+    """Only the prefilter's sample positions hold large values (the library
+    samples 128 evenly spread runs of 64 consecutive elements), so the
+    threshold estimate sits above the k-th magnitude and fewer than k elements
+    pass it: the rescan fallback must give the exact answer."""
     n, k = 4_000_000, 20_000
     g = np.full(n, 1e-6, np.float32)
-    m = 16384
-    sampled = (np.arange(m, dtype=np.int64) * n) // m
+    starts = (np.arange(128, dtype=np.int64) * n) >> 7
+    sampled = (starts[:, None] + np.arange(64)[None, :]).reshape(-1)
     mask = np.ones(n, bool)
     mask[sampled] = False
     pos = np.nonzero(mask)[0][::7][:50_000]
@@ -177,33 +178,3 @@ def test_bf16_ties_1p5b_full():
         assert same, f"step {step}: residuals differ"
     info = ef.topk_ef_path_info(ws)
     assert info["fallback"] == 0, info
-
-
-@pytest.mark.parametrize("n,k", [(8192 * 3, 30), (1_000_003, 1000), (4_000_001, 4000),
-                                 (25_557_032, 25_557)])
-def test_tma_staged_stream(n, k):
-    """The TMA-staged streaming kernel (test flag bit 2) gives the same
-    results, including partial last tiles and lengths not divisible by 4."""
-    rng = np.random.default_rng(n % 1000 + 5)
-    grads = [rng.laplace(0, 1e-3, n).astype(np.float32) for _ in range(2)]
-    old = ef.topk_ef_set_test_flags(4)
-    try:
-        run_compress_steps(grads, LR, k, backend=1, ws=_ws(n, k))
-    finally:
-        ef.topk_ef_set_test_flags(old)
-
-
-def test_tma_staged_batched():
-    sizes = [1, 7, 70_001, 8192, 3, 250_000, 5]
-    ks = [1, 3, 70, 8192, 0, 250, 5]
-    rng = np.random.default_rng(44)
-    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
-    grads = [rng.laplace(0, 1e-2, int(offsets[-1])).astype(np.float32) for _ in range(2)]
-    from gpu_util import run_batched_steps
-    ws = torch.empty(ef.topk_ef_batched_workspace_bytes(offsets, ks), dtype=torch.uint8,
-                     device="cuda")
-    old = ef.topk_ef_set_test_flags(4)
-    try:
-        run_batched_steps(grads, offsets, ks, LR, ws=ws)
-    finally:
-        ef.topk_ef_set_test_flags(old)
