@@ -72,6 +72,14 @@ class Oracle:
         lib.oracle_gtopk_merge.argtypes = [_i32p, _f32p, ctypes.c_int32, _i64, _i64,
                                            _i64, _i32p, _f32p]
         lib.oracle_gtopk_merge.restype = ctypes.c_int64
+        lib.oracle_threshold.argtypes = [_f32p, _f32p, _i64, ctypes.c_float, ctypes.c_float,
+                                         _i64, _i32p, _f32p]
+        lib.oracle_threshold.restype = ctypes.c_int64
+        lib.oracle_residual_return.argtypes = [_i32p, _f32p, ctypes.c_int32, _i64, _i32p,
+                                               _i64, _f32p, _i64]
+        lib.oracle_residual_return.restype = ctypes.c_int
+        lib.oracle_allgather_sum.argtypes = [_i32p, _f32p, ctypes.c_int32, _i64, _i64, _f32p]
+        lib.oracle_allgather_sum.restype = ctypes.c_int
         self._lib = lib
 
     # --- memory update -------------------------------------------------
@@ -140,6 +148,56 @@ class Oracle:
         if m < 0:
             raise ValueError(f"oracle_gtopk_merge failed: {m}")
         return oi[:m], ov[:m]
+
+
+    # --- hard threshold ----------------------------------------------------
+    def threshold(self, grad, residual, lr, threshold, max_out):
+        """Hard-threshold EF step: sends the first max_out (ascending index)
+        of the entries with |acc| >= |threshold|; residual updated in place.
+        Returns (idx, val, count) with count = all entries that passed."""
+        grad = np.ascontiguousarray(grad, dtype=np.float32)
+        assert residual.dtype == np.float32 and residual.flags.c_contiguous
+        max_out = int(max_out)
+        oi = np.empty(max(max_out, 1), dtype=np.int32)
+        ov = np.empty(max(max_out, 1), dtype=np.float32)
+        c = self._lib.oracle_threshold(grad, residual, grad.size, np.float32(lr),
+                                       np.float32(threshold), max_out, oi, ov)
+        if c < 0:
+            raise ValueError(f"oracle_threshold failed: {c}")
+        m = min(int(c), max_out)
+        return oi[:m], ov[:m], int(c)
+
+    # --- residual return after gTop-k ------------------------------------
+    def residual_return(self, sent_idx, sent_val, global_idx, residual):
+        """Adds back, per worker p (row of sent_*), the sent values whose
+        index is not in global_idx; residual is [P][n], updated in place."""
+        sent_idx = np.ascontiguousarray(sent_idx, dtype=np.int32)
+        sent_val = np.ascontiguousarray(sent_val, dtype=np.float32)
+        global_idx = np.ascontiguousarray(global_idx, dtype=np.int32)
+        assert residual.dtype == np.float32 and residual.flags.c_contiguous
+        P, k_sent = sent_idx.shape
+        n = residual.shape[-1]
+        si = sent_idx.reshape(-1) if sent_idx.size else np.zeros(1, np.int32)
+        sv = sent_val.reshape(-1) if sent_val.size else np.zeros(1, np.float32)
+        gi = global_idx if global_idx.size else np.zeros(1, np.int32)
+        rc = self._lib.oracle_residual_return(si, sv, P, k_sent, gi, global_idx.size,
+                                              residual.reshape(-1), n)
+        if rc != 0:
+            raise ValueError(f"oracle_residual_return failed: {rc}")
+
+    # --- AllGather aggregation ---------------------------------------------
+    def allgather_sum(self, in_idx, in_val, n):
+        """Dense sum of the P sets (rows), added in rank order from +0."""
+        in_idx = np.ascontiguousarray(in_idx, dtype=np.int32)
+        in_val = np.ascontiguousarray(in_val, dtype=np.float32)
+        P, k_in = in_idx.shape
+        out = np.empty(max(int(n), 1), dtype=np.float32)
+        fi = in_idx.reshape(-1) if in_idx.size else np.zeros(1, np.int32)
+        fv = in_val.reshape(-1) if in_val.size else np.zeros(1, np.float32)
+        rc = self._lib.oracle_allgather_sum(fi, fv, P, k_in, int(n), out)
+        if rc != 0:
+            raise ValueError(f"oracle_allgather_sum failed: {rc}")
+        return out[:int(n)]
 
 
 _default: Oracle | None = None

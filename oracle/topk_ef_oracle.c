@@ -434,3 +434,136 @@ done:
     free(chosen);
     return result;
 }
+
+/* ------------------------------------------------------------------------
+ * Hard-threshold sparsifier with error feedback.
+ * ("Rethinking gradient sparsification as total error minimization",
+ * abstract in the arxivdaily listing: the variant of Top-k in which k is set
+ * by a constant hard threshold, used under error feedback.)
+ *
+ *   acc          = fmaf(lr, grad, residual)
+ *   P            = { i : key(acc[i]) >= key(threshold) }   (|acc| at least |threshold|)
+ *   S            = the first min(|P|, max_out) members of P, ascending index
+ *   out          = (i, acc[i]) for i in S
+ *   residual[i]  = +0.0f for i in S, acc[i] otherwise
+ * Returns |P| (which may exceed max_out), or a negative error code.
+ * ---------------------------------------------------------------------- */
+int64_t oracle_threshold(const float *grad, float *residual, int64_t n,
+                         float lr, float threshold, int64_t max_out,
+                         int32_t *out_idx, float *out_val)
+{
+    if (n < 0 || max_out < 0 || n > 2147483647LL) return ORACLE_EINVAL;
+    if (n > 0 && (!grad || !residual)) return ORACLE_EINVAL;
+    if (max_out > 0 && (!out_idx || !out_val)) return ORACLE_EINVAL;
+    if (n == 0) return 0;
+    float *acc = (float *)malloc((size_t)n * sizeof(float));
+    if (!acc) return ORACLE_ENOMEM;
+    oracle_accumulate(grad, residual, n, lr, acc);
+    const uint32_t t = key_of(threshold);
+    int64_t passed = 0;
+    for (int64_t i = 0; i < n; ++i) {
+        residual[i] = acc[i];
+#if ORACLE_MUTANT == 10
+        /* mistake: strictly above the threshold */
+        int in = key_of(acc[i]) > t;
+#else
+        int in = key_of(acc[i]) >= t;
+#endif
+        if (!in) continue;
+        if (passed < max_out) {
+            out_idx[passed] = (int32_t)i;
+            out_val[passed] = acc[i];
+            residual[i] = 0.0f;
+        }
+        ++passed;
+    }
+    free(acc);
+    return passed;
+}
+
+/* ------------------------------------------------------------------------
+ * gTop-k residual return.
+ * (Error feedback, "Sparsified SGD with Memory" and "The Convergence of
+ * Sparsified Gradient Methods", abstracts: what is not transmitted stays in
+ * local memory; "A Distributed Synchronous SGD Algorithm with Global Top-k
+ * Sparsification", ABSTRACT: only the global top-k of the P workers' values
+ * updates the model.)  A value that worker p sent but whose index is not in
+ * the global set was not transmitted in effect, so it goes back to p's
+ * memory:
+ *     for p, j:  i = sent_idx[p][j];  if i is not in global_idx[0..k_global):
+ *                    residual[p][i] = residual[p][i] + sent_val[p][j]
+ * (one fp32 add).  residual is [P][n].  Rows of sent_idx ascend strictly.
+ * ---------------------------------------------------------------------- */
+int oracle_residual_return(const int32_t *sent_idx, const float *sent_val,
+                           int32_t P, int64_t k_sent,
+                           const int32_t *global_idx, int64_t k_global,
+                           float *residual, int64_t n)
+{
+    if (P < 1 || k_sent < 0 || k_global < 0 || n < 0 || n > 2147483647LL)
+        return ORACLE_EINVAL;
+    if ((k_sent > 0 && (!sent_idx || !sent_val)) || (k_global > 0 && !global_idx))
+        return ORACLE_EINVAL;
+    if (n > 0 && !residual) return ORACLE_EINVAL;
+    uint8_t *in_global = (uint8_t *)calloc((size_t)(n > 0 ? n : 1), 1);
+    if (!in_global) return ORACLE_ENOMEM;
+    for (int64_t j = 0; j < k_global; ++j) {
+        int32_t i = global_idx[j];
+        if (i < 0 || (int64_t)i >= n) { free(in_global); return ORACLE_EINVAL; }
+        in_global[i] = 1;
+    }
+    for (int32_t p = 0; p < P; ++p)
+        for (int64_t j = 0; j < k_sent; ++j) {
+            int32_t i = sent_idx[(int64_t)p * k_sent + j];
+            if (i < 0 || (int64_t)i >= n) { free(in_global); return ORACLE_EINVAL; }
+        }
+    for (int32_t p = 0; p < P; ++p) {
+        float *r = residual + (int64_t)p * n;
+        for (int64_t j = 0; j < k_sent; ++j) {
+            int32_t i = sent_idx[(int64_t)p * k_sent + j];
+#if ORACLE_MUTANT == 11
+            /* mistake: returns the values that did survive */
+            if (!in_global[i]) continue;
+#else
+            if (in_global[i]) continue;
+#endif
+            r[i] = r[i] + sent_val[(int64_t)p * k_sent + j];
+        }
+    }
+    free(in_global);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------
+ * Top-k aggregation by AllGather (the O(kP) TopKAllReduce that the gTop-k
+ * review compares against: "A Distributed Synchronous SGD Algorithm with
+ * Global Top-k Sparsification", ABSTRACT: current methods use AllGather to
+ * accumulate the sparse gradients).  Every worker receives all P local
+ * top-k sets and sums them into a dense gradient, in rank order:
+ *     out[i] = +0.0f for all i;  for p = 0..P-1, for each (i, v) in S_p:
+ *         out[i] = out[i] + v            (one fp32 add each)
+ * ---------------------------------------------------------------------- */
+int oracle_allgather_sum(const int32_t *in_idx, const float *in_val,
+                         int32_t P, int64_t k_in, int64_t n, float *out)
+{
+    if (P < 1 || k_in < 0 || n < 0 || k_in > n || n > 2147483647LL) return ORACLE_EINVAL;
+    if (k_in > 0 && (!in_idx || !in_val)) return ORACLE_EINVAL;
+    if (n > 0 && !out) return ORACLE_EINVAL;
+    for (int32_t p = 0; p < P; ++p)
+        for (int64_t j = 0; j < k_in; ++j) {
+            int32_t i = in_idx[(int64_t)p * k_in + j];
+            if (i < 0 || (int64_t)i >= n) return ORACLE_EINVAL;
+            if (j > 0 && in_idx[(int64_t)p * k_in + j - 1] >= i) return ORACLE_EINVAL;
+        }
+    for (int64_t i = 0; i < n; ++i) out[i] = 0.0f;
+#if ORACLE_MUTANT == 12
+    /* mistake: reverse rank order */
+    for (int32_t p = P - 1; p >= 0; --p)
+#else
+    for (int32_t p = 0; p < P; ++p)
+#endif
+        for (int64_t j = 0; j < k_in; ++j) {
+            int32_t i = in_idx[(int64_t)p * k_in + j];
+            out[i] = out[i] + in_val[(int64_t)p * k_in + j];
+        }
+    return ORACLE_OK;
+}

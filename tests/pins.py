@@ -14,7 +14,13 @@ the oracle with a planted mistake must fail at least one
 * special cases (k = 0, k = n, lr = 1 with zero memory, all magnitudes equal);
 * hand-worked examples under tests/golden/ (one EF run, one merge tournament);
 * merge special cases: P = 1 identity, disjoint supports give the plain union,
-  and with k >= |union| the tournament is the dense pairwise tree sum.
+  and with k >= |union| the tournament is the dense pairwise tree sum;
+* hard threshold: hand-worked run, special thresholds (0, +Inf, a negative
+  threshold, max_out = 0) and agreement with the top-k step at k = count;
+* residual return: hand-worked example, a global set that holds every sent
+  index (nothing returned) and one that holds none (everything returned);
+* AllGather sum: hand-worked example (rank order visible in fp32), and on
+  values whose sums are exact it equals the gTop-k merge with k >= |union|.
 """
 from __future__ import annotations
 
@@ -348,10 +354,127 @@ def _dominates_all_ids(v, ids, S):
     return True
 
 
+# ------------------------------------------------------------ hard threshold
+
+def pin_golden_threshold(o):
+    with open(os.path.join(GOLDEN, "threshold_small.json")) as f:
+        g = json.load(f)
+    r = np.array(g["residual0"], np.float32)
+    for st in g["steps"]:
+        idx, val, cnt = o.threshold(np.array(st["grad"], np.float32), r, g["lr"],
+                                    g["threshold"], g["max_out"])
+        assert cnt == st["count"], (cnt, st["count"])
+        assert idx.tolist() == st["idx"], (idx, st["idx"])
+        assert val.tolist() == st["val"], (val, st["val"])
+        assert r.tolist() == st["residual"], (r, st["residual"])
+
+
+def pin_threshold_special(o, seed=21):
+    rng = np.random.default_rng(seed)
+    n = 300
+    grad = rng.standard_normal(n).astype(np.float32)
+    res = (rng.standard_normal(n) * 0.5).astype(np.float32)
+    acc = _exact_acc(grad, res, np.float32(0.5))
+    # threshold 0: every entry passes; the first max_out are sent
+    r = res.copy()
+    idx, val, cnt = o.threshold(grad, r, 0.5, 0.0, 40)
+    assert cnt == n and idx.tolist() == list(range(40))
+    assert np.array_equal(_bits(val), _bits(acc[:40]))
+    assert np.all(_bits(r[:40]) == 0) and np.array_equal(_bits(r[40:]), _bits(acc[40:]))
+    # max_out = 0: nothing sent, the count is still reported
+    r = res.copy()
+    idx, val, cnt = o.threshold(grad, r, 0.5, 0.0, 0)
+    assert cnt == n and idx.size == 0 and np.array_equal(_bits(r), _bits(acc))
+    # +Inf: only infinities and NaNs pass; a negative threshold acts by magnitude
+    x = np.array([1.0, -np.inf, 3.0, np.nan, np.inf, -3.0], np.float32)
+    z = np.zeros(6, np.float32)
+    idx, val, cnt = o.threshold(x, z.copy(), 1.0, np.inf, 10)
+    assert cnt == 3 and idx.tolist() == [1, 3, 4]
+    idx, val, cnt = o.threshold(x, z.copy(), 1.0, -3.0, 10)
+    assert idx.tolist() == [1, 2, 3, 4, 5]
+
+
+def pin_threshold_matches_topk(o, seed=22):
+    """With room for every passing entry, the sent set is the top-k set for
+    k = count (nothing outside it has a magnitude at or above the threshold),
+    so the two steps agree bit for bit."""
+    rng = np.random.default_rng(seed)
+    for n, thr in ((5_000, 1.5), (20_000, 2.5), (777, 0.25)):
+        grad = rng.standard_normal(n).astype(np.float32)
+        res = (rng.standard_normal(n) * 0.1).astype(np.float32)
+        at = rng.integers(0, n, n // 10)
+        grad[at] = np.float32(thr) * 2          # acc = 0.5 * 2 thr exactly at the threshold
+        res[at] = 0.0
+        r1, r2 = res.copy(), res.copy()
+        idx, val, cnt = o.threshold(grad, r1, 0.5, thr, n)
+        ti, tv = o.compress(grad, r2, 0.5, cnt)
+        assert np.array_equal(idx, ti) and np.array_equal(_bits(val), _bits(tv))
+        assert np.array_equal(_bits(r1), _bits(r2))
+
+
+# ----------------------------------------------------------- residual return
+
+def pin_golden_residual_return(o):
+    with open(os.path.join(GOLDEN, "residual_return_small.json")) as f:
+        g = json.load(f)
+    r = np.array(g["residual0"], np.float32)
+    o.residual_return(np.array(g["sent_idx"], np.int32), np.array(g["sent_val"], np.float32),
+                      np.array(g["global_idx"], np.int32), r)
+    assert r.tolist() == g["residual"], (r, g["residual"])
+
+
+def pin_residual_return_special(o, seed=23):
+    rng = np.random.default_rng(seed)
+    P, k, n = 4, 50, 1000
+    idx = np.stack([np.sort(rng.choice(n, k, replace=False)) for _ in range(P)]).astype(np.int32)
+    val = rng.standard_normal((P, k)).astype(np.float32)
+    res = rng.standard_normal((P, n)).astype(np.float32)
+    # every sent index survived: nothing comes back
+    r = res.copy()
+    o.residual_return(idx, val, np.unique(idx).astype(np.int32), r)
+    assert np.array_equal(_bits(r), _bits(res))
+    # no sent index survived: every sent value comes back (memory was +0 there)
+    r = res.copy()
+    for p in range(P):
+        r[p, idx[p]] = 0.0
+    want = r.copy()
+    for p in range(P):
+        want[p, idx[p]] = val[p]
+    rest = np.setdiff1d(np.arange(n), np.unique(idx))[:30].astype(np.int32)
+    o.residual_return(idx, val, rest, r)
+    assert np.array_equal(_bits(r), _bits(want))
+
+
+# ------------------------------------------------------------ AllGather sum
+
+def pin_golden_allgather(o):
+    with open(os.path.join(GOLDEN, "allgather_small.json")) as f:
+        g = json.load(f)
+    out = o.allgather_sum(np.array(g["idx"], np.int32), np.array(g["val"], np.float32), g["n"])
+    assert out.tolist() == g["out"], (out, g["out"])
+
+
+def pin_allgather_matches_merge(o, seed=24):
+    """Small integer values add exactly in any order, so the dense sum equals
+    the gTop-k tournament kept whole (k >= |union|) scattered into zeros."""
+    rng = np.random.default_rng(seed)
+    for P, k, n in ((5, 40, 200), (8, 100, 5000), (1, 10, 10)):
+        idx = np.stack([np.sort(rng.choice(n, k, replace=False)) for _ in range(P)]).astype(np.int32)
+        val = rng.integers(-50, 51, (P, k)).astype(np.float32)
+        dense = o.allgather_sum(idx, val, n)
+        mi, mv = o.gtopk_merge(idx, val, P * k, n)
+        want = np.zeros(n, np.float32)
+        want[mi] = mv
+        assert np.array_equal(dense, want)
+        assert np.count_nonzero(np.isin(np.arange(n), mi)) == np.unique(idx).size
+
+
 ALL_PINS = [
     pin_fmaf_exact, pin_bruteforce_select, pin_compress_invariants,
     pin_special_cases, pin_backends_agree, pin_golden_compress,
     pin_batched_matches_flat, pin_golden_merge, pin_merge_identity,
     pin_merge_disjoint_union, pin_merge_dense_tree_sum,
-    pin_merge_bruteforce_select,
+    pin_merge_bruteforce_select, pin_golden_threshold, pin_threshold_special,
+    pin_threshold_matches_topk, pin_golden_residual_return,
+    pin_residual_return_special, pin_golden_allgather, pin_allgather_matches_merge,
 ]

@@ -6,14 +6,15 @@ The mistakes are compiled into copies of the oracle on the CPU
  3 signed instead of |x| order  4 fma operands transposed
  5 sent value left in memory    6 partner value dropped in the merge
  7 merge partner ignores round  8 output not in index order
- 9 two roundings instead of one
+ 9 two roundings instead of one  10 hard threshold strictly above
+11 residual return inverted      12 AllGather sum in reverse rank order
 """
 import pytest
 
 import oracle
 import pins
 
-MUTANTS = list(range(1, 10))
+MUTANTS = list(range(1, 13))
 
 
 @pytest.mark.parametrize("m", MUTANTS)
