@@ -312,7 +312,7 @@ class Merge:
         merges = P - 1
         self.bytes_per_step = merges * 3 * 8 * k
         self.elems_per_step = P * k
-        self.dominant = "merge_round_kernel"
+        self.dominant = "merge_cluster_kernel"
         self.dominant_bytes = None
         self.flush = True
         self.rounds = rounds
@@ -363,6 +363,151 @@ class Merge:
         return {}
 
 
+class ThresholdCompress:
+    """One hard-threshold EF step (topk_ef_threshold) on the ResNet-50-sized
+    mixed gradient, threshold 6e-3 (about 0.1% pass at the first step),
+    max_out = 1% of n."""
+
+    def __init__(self, thr=6e-3):
+        self.n = datagen.RESNET50_N
+        self.thr = thr
+        self.max_out = self.n // 100
+        self.elems_per_step = self.n
+        self.dominant = "stream_kernel"
+        self.dominant_bytes = 12 * self.n
+        self.flush = False
+        self.bytes_per_step = 12 * self.n      # + 8 per sent pair, set after warm-up
+
+    def config(self):
+        return {"workload": f"hard_threshold: resnet50_mix n={self.n:,}, |acc| >= {self.thr}, "
+                            f"max_out={self.max_out:,}", "n": self.n, "lr": float(LR),
+                "l2": l2_note(self.flush, 8 * self.n),
+                "parallelism": "replicas (one independent EF step per GPU)"}
+
+    def setup(self, rank, steps_needed):
+        import torch
+        import error_feedback_b200 as ef
+        self.ef = ef
+        npool = min(POOL, max(1, steps_needed))
+        host = [datagen.resnet50_mix(100 * rank + s) for s in range(npool)]
+        self.dev = [torch.from_numpy(g).cuda() for g in host]
+        self.hpin = [torch.from_numpy(g).pin_memory() for g in host]
+        self.res = torch.zeros(self.n, dtype=torch.float32, device="cuda")
+        self.oi = torch.empty(self.max_out, dtype=torch.int32, device="cuda")
+        self.ov = torch.empty(self.max_out, dtype=torch.float32, device="cuda")
+        self.oc = torch.empty(1, dtype=torch.int64, device="cuda")
+        self.ws = torch.empty(ef.topk_ef_threshold_workspace_bytes(self.n), dtype=torch.uint8,
+                              device="cuda")
+        self.stage = torch.empty(self.n, dtype=torch.float32, device="cuda")
+        self.hoi = torch.empty(self.max_out, dtype=torch.int32).pin_memory()
+        self.hov = torch.empty(self.max_out, dtype=torch.float32).pin_memory()
+        self.hoc = torch.empty(1, dtype=torch.int64).pin_memory()
+        self.h2d_bytes = 4 * self.n
+        self.d2h_bytes = 8 * self.max_out + 8
+
+    def after_warmup(self):
+        sent = min(int(self.oc.cpu().item()), self.max_out)
+        self.bytes_per_step = 12 * self.n + 8 * sent
+        self.sent = sent
+
+    def step(self, i):
+        self.ef.topk_ef_threshold(self.dev[i % len(self.dev)], self.res, LR, self.thr,
+                                  self.max_out, self.oi, self.ov, self.oc, self.ws)
+
+    def e2e_step(self, i):
+        self.stage.copy_(self.hpin[i % len(self.hpin)], non_blocking=True)
+        self.ef.topk_ef_threshold(self.stage, self.res, LR, self.thr, self.max_out, self.oi,
+                                  self.ov, self.oc, self.ws)
+        self.hoc.copy_(self.oc, non_blocking=True)
+        self.hoi.copy_(self.oi, non_blocking=True)
+        self.hov.copy_(self.ov, non_blocking=True)
+
+    def status(self):
+        return self.ef.topk_ef_last_device_status(self.ws)
+
+    def path(self):
+        return {"sent_per_step_after_warmup": getattr(self, "sent", None)}
+
+
+class SparseAfterMerge:
+    """The steps around the gTop-k merge on its configuration (P = 32 sets of
+    k = 25,557 over n = 25,557,032): the residual return of the non-surviving
+    sent values to all 32 workers' memories ([32][n] fp32), or the AllGather
+    dense rank-order sum of all sets."""
+
+    def __init__(self, kind, P=32, k=25_557, n=datagen.RESNET50_N):
+        self.kind, self.P, self.k, self.n = kind, P, k, n
+        self.elems_per_step = P * k
+        self.flush = True
+        self.dominant = "return_kernel" if kind == "return" else "ag_sum_kernel"
+
+    def config(self):
+        what = ("gtopk_residual_return: 32 workers' memories [32][n]" if self.kind == "return"
+                else "topk_allgather_sum: dense rank-order sum of 32 sets")
+        return {"workload": f"{what}, P={self.P} k={self.k} n={self.n}", "P": self.P,
+                "k": self.k, "n": self.n,
+                "l2": "flushed between steps (256 MiB write, not timed)",
+                "parallelism": "P workers simulated on each GPU"}
+
+    def setup(self, rank, steps_needed):
+        import torch
+        import error_feedback_b200 as ef
+        self.ef = ef
+        idx, val = datagen.gtopk_sets(P=self.P, k=self.k, n=self.n, step=rank)
+        self.di = torch.from_numpy(idx).cuda()
+        self.dv = torch.from_numpy(val).cuda()
+        self.hi = torch.from_numpy(idx).pin_memory()
+        self.hv = torch.from_numpy(val).pin_memory()
+        self.si = torch.empty_like(self.di)
+        self.sv = torch.empty_like(self.dv)
+        if self.kind == "return":
+            gi = torch.empty(self.k, dtype=torch.int32, device="cuda")
+            gv = torch.empty(self.k, dtype=torch.float32, device="cuda")
+            gc = torch.empty(1, dtype=torch.int32, device="cuda")
+            ef.gtopk_merge(self.di, self.dv, self.k, self.n, gi, gv, gc)
+            self.gidx = gi[:int(gc.cpu().item())].contiguous()
+            self.res = torch.zeros((self.P, self.n), dtype=torch.float32, device="cuda")
+            self.ws = torch.empty(ef.gtopk_residual_return_workspace_bytes(), dtype=torch.uint8,
+                                  device="cuda")
+            returned = int((~np.isin(idx, self.gidx.cpu().numpy())).sum())
+            # read the sent sets and the global list, read and write each returned value
+            self.bytes_per_step = 8 * self.P * self.k + 4 * self.gidx.numel() + 8 * returned
+            self.h2d_bytes = 8 * self.P * self.k
+            self.d2h_bytes = 0
+        else:
+            self.out = torch.empty(self.n, dtype=torch.float32, device="cuda")
+            self.hout = torch.empty(self.n, dtype=torch.float32).pin_memory()
+            self.ws = torch.empty(ef.topk_allgather_workspace_bytes(self.P, self.k, self.n),
+                                  dtype=torch.uint8, device="cuda")
+            # read the sets, write the dense sum
+            self.bytes_per_step = 8 * self.P * self.k + 4 * self.n
+            self.h2d_bytes = 8 * self.P * self.k
+            self.d2h_bytes = 4 * self.n
+        self.dominant_bytes = self.bytes_per_step
+
+    def _run(self, i, si, sv):
+        if self.kind == "return":
+            self.ef.gtopk_residual_return(si, sv, self.gidx, self.res, ws=self.ws)
+        else:
+            self.ef.topk_allgather_sum(si, sv, self.n, out=self.out, ws=self.ws)
+
+    def step(self, i):
+        self._run(i, self.di, self.dv)
+
+    def e2e_step(self, i):
+        self.si.copy_(self.hi, non_blocking=True)
+        self.sv.copy_(self.hv, non_blocking=True)
+        self._run(i, self.si, self.sv)
+        if self.kind != "return":
+            self.hout.copy_(self.out, non_blocking=True)
+
+    def status(self):
+        return self.ef.topk_ef_last_device_status(self.ws)
+
+    def path(self):
+        return {}
+
+
 def make_workload(name):
     n3 = datagen.RESNET50_N
     if name in ("resnet50_mix", "resnet50_mix_0.1pct"):
@@ -385,6 +530,12 @@ def make_workload(name):
         return BatchedCompress()
     if name == "gtopk_merge_p32":
         return Merge()
+    if name == "hard_threshold_resnet50":
+        return ThresholdCompress()
+    if name == "gtopk_return_p32":
+        return SparseAfterMerge("return")
+    if name == "allgather_sum_p32":
+        return SparseAfterMerge("allgather")
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -418,6 +569,8 @@ def run_ours(args):
     st = wl.status()
     if st != 0:
         raise SystemExit(f"device status after warm-up: {ef.status_string(st)}")
+    if hasattr(wl, "after_warmup"):
+        wl.after_warmup()
 
     # launches per step and per-kernel times: a short fully traced run before
     # the timed region (tracing every launch breaks the overlap between them)
@@ -563,6 +716,38 @@ def time_oracle(wl, steps, budget_elems):
             o.gtopk_merge(idx, val, wl.k, wl.nidx)
         dt = time.perf_counter() - t0
         return dt, f"{steps} full tournaments", wl.bytes_per_step, wl.elems_per_step
+    if isinstance(wl, ThresholdCompress):
+        ns = int(min(wl.n, budget_elems or wl.n))
+        g = datagen.resnet50_mix(0)[:ns].copy()
+        res = np.zeros(ns, np.float32)
+        t0 = time.perf_counter()
+        sent = 0
+        for _ in range(steps):
+            _, _, c = o.threshold(g, res, LR, wl.thr, ns // 100)
+            sent += min(c, ns // 100)
+        dt = time.perf_counter() - t0
+        return (dt, f"{steps} hard-threshold steps on the first {ns} elements",
+                12 * ns + 8 * sent // max(1, steps), ns)
+    if isinstance(wl, SparseAfterMerge):
+        idx, val = datagen.gtopk_sets(P=wl.P, k=wl.k, n=wl.n)
+        if wl.kind == "return":
+            gi, _ = o.gtopk_merge(idx, val, wl.k, wl.n)
+            rows = 4                     # memories of 4 of the 32 workers (host RAM)
+            res = np.zeros((rows, wl.n), np.float32)
+            t0 = time.perf_counter()
+            for _ in range(steps):
+                o.residual_return(idx[:rows], val[:rows], gi, res)
+            dt = time.perf_counter() - t0
+            frac = rows / wl.P
+            return (dt, f"{steps} residual returns to {rows} of the {wl.P} workers",
+                    wl.bytes_per_step * frac if hasattr(wl, "bytes_per_step") else 8 * rows * wl.k,
+                    rows * wl.k)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            o.allgather_sum(idx, val, wl.n)
+        dt = time.perf_counter() - t0
+        return (dt, f"{steps} dense sums of all {wl.P} sets", 8 * wl.P * wl.k + 4 * wl.n,
+                wl.elems_per_step)
     raise SystemExit("no oracle sample for this workload")
 
 

@@ -64,6 +64,20 @@ def lib() -> ctypes.CDLL:
         L.topk_ef_compress_static.argtypes = [_vp, _vp, _i64, ctypes.c_float, _i64, _vp, _vp,
                                               _vp]
         L.topk_ef_compress_static.restype = ctypes.c_int
+        L.topk_ef_threshold_workspace_bytes.argtypes = [_i64]
+        L.topk_ef_threshold_workspace_bytes.restype = _sz
+        L.topk_ef_threshold.argtypes = [_vp, _vp, _i64, ctypes.c_float, ctypes.c_float, _i64,
+                                        _vp, _vp, _vp, _vp, _sz, _vp]
+        L.topk_ef_threshold.restype = ctypes.c_int
+        L.gtopk_residual_return_workspace_bytes.argtypes = []
+        L.gtopk_residual_return_workspace_bytes.restype = _sz
+        L.gtopk_residual_return.argtypes = [_vp, _vp, _i32, _i64, _vp, _i64, _vp, _i64, _vp,
+                                            _sz, _vp]
+        L.gtopk_residual_return.restype = ctypes.c_int
+        L.topk_allgather_workspace_bytes.argtypes = [_i32, _i64, _i64]
+        L.topk_allgather_workspace_bytes.restype = _sz
+        L.topk_allgather_sum.argtypes = [_vp, _vp, _i32, _i64, _i64, _vp, _vp, _sz, _vp]
+        L.topk_allgather_sum.restype = ctypes.c_int
         L.topk_ef_batched_workspace_bytes.argtypes = [_pi64, _pi64, _i32]
         L.topk_ef_batched_workspace_bytes.restype = _sz
         L.topk_ef_compress_batched.argtypes = [_vp, _vp, _pi64, _pi64, _i32, ctypes.c_float, _vp, _vp,
@@ -182,6 +196,92 @@ def topk_ef_compress_static(grad, residual, lr, k, out_idx=None, out_val=None, s
                                        out_idx.data_ptr(), out_val.data_ptr(), _stream(stream))
     _check(rc, "topk_ef_compress_static")
     return out_idx, out_val
+
+
+def topk_ef_threshold_workspace_bytes(n: int) -> int:
+    return int(lib().topk_ef_threshold_workspace_bytes(int(n)))
+
+
+def topk_ef_threshold(grad, residual, lr, threshold, max_out, out_idx=None, out_val=None,
+                      out_count=None, ws=None, stream=None):
+    """Hard-threshold EF step: acc = fmaf(lr, grad, residual); the entries
+    with |acc| >= |threshold| pass and the first max_out of them (ascending
+    index) are sent, their residual zeroed.  Returns (idx int32[max_out],
+    val float32[max_out], count int64[1] on the device); only the first
+    min(count, max_out) slots of idx / val are written."""
+    _cuda_f32(grad, "grad")
+    _cuda_f32(residual, "residual")
+    if grad.numel() != residual.numel():
+        raise ValueError("grad and residual differ in size")
+    n, max_out = grad.numel(), int(max_out)
+    dev = grad.device
+    if out_idx is None:
+        out_idx = torch.empty(max(max_out, 1), dtype=torch.int32, device=dev)[:max_out]
+    if out_val is None:
+        out_val = torch.empty(max(max_out, 1), dtype=torch.float32, device=dev)[:max_out]
+    if out_count is None:
+        out_count = torch.empty(1, dtype=torch.int64, device=dev)
+    nb = topk_ef_threshold_workspace_bytes(n)
+    if nb == 0:
+        raise TopkEfError(ERR_INVALID_ARG, "topk_ef_threshold_workspace_bytes")
+    ws = _workspace(nb, dev, ws)
+    rc = lib().topk_ef_threshold(grad.data_ptr(), residual.data_ptr(), n, float(lr),
+                                 float(threshold), max_out, out_idx.data_ptr(),
+                                 out_val.data_ptr(), out_count.data_ptr(), ws.data_ptr(),
+                                 ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "topk_ef_threshold")
+    return out_idx, out_val, out_count
+
+
+def gtopk_residual_return_workspace_bytes() -> int:
+    return int(lib().gtopk_residual_return_workspace_bytes())
+
+
+def gtopk_residual_return(sent_idx, sent_val, global_idx, residual, ws=None, stream=None):
+    """After gTop-k: for every worker p (row of sent_idx / sent_val) and sent
+    (i, v) with i not in global_idx, residual[p, i] += v.  residual is a
+    [P, n] float32 CUDA tensor, updated in place."""
+    for t, name in ((sent_idx, "sent_idx"), (global_idx, "global_idx")):
+        if not t.is_cuda or t.dtype != torch.int32 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous int32 CUDA tensor")
+    _cuda_f32(sent_val, "sent_val")
+    _cuda_f32(residual, "residual")
+    P, k_sent = sent_idx.shape
+    if residual.dim() != 2 or residual.shape[0] != P or tuple(sent_val.shape) != (P, k_sent):
+        raise ValueError("shapes: sent_idx/sent_val [P, k_sent], residual [P, n]")
+    n = residual.shape[1]
+    ws = _workspace(gtopk_residual_return_workspace_bytes(), residual.device, ws)
+    rc = lib().gtopk_residual_return(sent_idx.data_ptr(), sent_val.data_ptr(), P, k_sent,
+                                     global_idx.data_ptr(), global_idx.numel(),
+                                     residual.data_ptr(), n, ws.data_ptr(),
+                                     ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "gtopk_residual_return")
+    return ws
+
+
+def topk_allgather_workspace_bytes(P: int, k_in: int, n: int) -> int:
+    return int(lib().topk_allgather_workspace_bytes(int(P), int(k_in), int(n)))
+
+
+def topk_allgather_sum(in_idx, in_val, n, out=None, ws=None, stream=None):
+    """Dense rank-order sum of the P sets (rows of in_idx / in_val) into a
+    float32[n] CUDA tensor (the AllGather aggregation)."""
+    if not in_idx.is_cuda or in_idx.dtype != torch.int32 or not in_idx.is_contiguous():
+        raise TypeError("in_idx must be a contiguous int32 CUDA tensor")
+    _cuda_f32(in_val, "in_val")
+    P, k_in = in_idx.shape
+    n = int(n)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=torch.float32, device=in_idx.device)[:n]
+    nb = topk_allgather_workspace_bytes(P, k_in, n)
+    if nb == 0:
+        raise TopkEfError(ERR_INVALID_ARG, "topk_allgather_workspace_bytes")
+    ws = _workspace(nb, in_idx.device, ws)
+    rc = lib().topk_allgather_sum(in_idx.data_ptr(), in_val.data_ptr(), P, k_in, n,
+                                  out.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                  _stream(stream))
+    _check(rc, "topk_allgather_sum")
+    return out
 
 
 def topk_ef_batched_workspace_bytes(offsets, k) -> int:

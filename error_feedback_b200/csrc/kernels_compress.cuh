@@ -65,6 +65,8 @@ struct SetupParams {
     uint32_t r[TCAP];       // target rank among the samples
     uint32_t r_hi[TCAP];    // rank of an upper estimate of the k-th key
     uint16_t sampled[TCAP]; // i-th sampled tensor (block i samples it)
+    int32_t has_fixed_T0;   // hard threshold: every tensor uses fixed_T0
+    uint32_t fixed_T0;
 };
 
 // Block i < n_sampled samples acc for the prefilter threshold T0 of the i-th
@@ -180,7 +182,7 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
             sm.n = p.off[l + 1] - p.off[l];
             sm.out_base = p.out_base[l];
             sm.k = p.k[l];
-            sm.T0 = p.k[l] == 0 ? NO_KEY : 0u;
+            sm.T0 = p.has_fixed_T0 ? p.fixed_T0 : (p.k[l] == 0 ? NO_KEY : 0u);
             sm.shift = REL_MAX_SHIFT;
             p.meta[l] = sm;
         }

@@ -440,7 +440,10 @@ __device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, 
 // offset) from position pos of the dense list, and add each to the relative
 // digit-1 histogram of its tensor: s_r1 (shared) when the caller's chunk
 // lies in tensor lc, else the global one.  S.seg holds element offsets.
-template <int C>
+// In threshold mode (kThr) the dense list is the caller's output: a written
+// candidate is sent, so its residual becomes +0.0f, and there is no
+// histogram.
+template <int C, bool kThr>
 __device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelShared& S,
                                              uint32_t w, uint64_t pos, uint32_t cnt,
                                              const TileCands& t, uint32_t* s_r1, int lc) {
@@ -456,8 +459,9 @@ __device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelSh
         if (q < src.cap) {
             src.cand_idx[q] = (uint32_t)e;
             src.cand_val[q] = t.v[i];
+            if (kThr) src.resid[e] = 0.0f;
         }
-        r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), t.v[i], s_r1);
+        if (!kThr) r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), t.v[i], s_r1);
     }
 }
 
@@ -489,41 +493,46 @@ __device__ uint64_t look_back(const uint64_t* agg, int c, uint32_t* status, SelS
 }
 
 // Gather a warp tile with more than WT_CAP candidates (one warp): rescan it
-// from the residual (which holds acc) with the streaming pass's test.
+// from the residual (which holds acc) with the streaming pass's test.  The
+// 32 coalesced loads of the tile (element base + 32 u + lane) are issued at
+// once; one ballot per load gives the positions in index order.
+template <bool kThr>
 __device__ void gather_rescan(const CompressSrc& src, const SelShared& S, uint32_t w,
                               uint64_t pos, uint32_t* s_r1, int lc) {
-    constexpr int U = 8;
     const uint32_t lane = lane_id();
     const int T = src.T;
     const int64_t base = (int64_t)w * WT;
     const int64_t tend = min(base + (int64_t)WT, src.N);
-    for (int64_t e0 = base; e0 < tend; e0 += 32 * U) {
-        float v[U];
+    float v[32];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t e = e0 + 32 * u + lane;
-            v[u] = e < tend ? src.resid[e] : 0.f;
-        }
+    for (int u = 0; u < 32; ++u) {
+        const int64_t e = base + 32 * u + lane;
+        v[u] = e < tend ? src.resid[e] : 0.f;
+    }
+    // tensor of each element: walk forward from the lane's first element
+    int l = lc;
+    if (!s_r1 && base + (int64_t)lane < tend) l = seg_of(S.seg, T, base + lane);
+    const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t e = e0 + 32 * u + lane;
-            bool f = false;
-            int l = lc;
-            if (e < tend) {
-                if (!s_r1) l = seg_of(S.seg, T, e);
-                f = key_of(v[u]) >= S.T0[l];
-            }
-            const uint32_t m = __ballot_sync(0xFFFFFFFFu, f);
-            if (f) {
-                const uint64_t q = pos + __popc(m & ((1u << lane) - 1u));
-                if (q < src.cap) {
-                    src.cand_idx[q] = (uint32_t)e;
-                    src.cand_val[q] = v[u];
-                }
-                r1_add(src, S, l, v[u], s_r1);
-            }
-            pos += __popc(m);
+    for (int u = 0; u < 32; ++u) {
+        const int64_t e = base + 32 * u + lane;
+        bool f = false;
+        if (e < tend) {
+            if (!s_r1)
+                while (l < T - 1 && S.seg[l + 1] <= e) ++l;
+            f = key_of(v[u]) >= S.T0[l];
         }
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, f);
+        if (f) {
+            const uint64_t q = pos + __popc(m & lt);
+            if (q < src.cap) {
+                src.cand_idx[q] = (uint32_t)e;
+                src.cand_val[q] = v[u];
+                if (kThr) src.resid[e] = 0.0f;
+            }
+            if (!kThr) r1_add(src, S, l, v[u], s_r1);
+        }
+        pos += __popc(m);
     }
 }
 
@@ -548,13 +557,11 @@ __device__ uint32_t tile_count_below(const CompressSrc& src, const SelShared& S,
 // barrier).  It copies its candidates, in index order, to [my0, my1) of the
 // dense list (the staged ones from registers loaded before the look-back;
 // tiles with more than WT_CAP candidates are rescanned), builds the relative
-// digit-1 histograms and records where each tensor's candidates start.
-// After one grid barrier every block takes the same decision: candidates
-// only if the list fit and each tensor kept at least k of them with its
-// k-th key inside the range of the relative digits.  Returns false if a
-// barrier gave up.
-__device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
-                                SelShared& S, uint64_t& my0, uint64_t& my1) {
+// digit-1 histograms (not in threshold mode) and records where each
+// tensor's candidates start.
+template <bool kThr>
+__device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S, uint64_t& my0,
+                             uint64_t& my1) {
     const int G = gridDim.x, c = blockIdx.x, tid = threadIdx.x;
     const uint32_t warp = warp_id(), nwarps = blockDim.x >> 5;
     const int T = src.T;
@@ -581,7 +588,7 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
     // relative digit 1 in shared memory when the whole chunk is in one tensor
     const int64_t e0 = (int64_t)w0 * WT, e1 = min((int64_t)w1 * WT, src.N);
     const int lc = w0 < w1 ? seg_of(s_off, T, e0) : 0;
-    const bool one = w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
+    const bool one = !kThr && w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
     uint32_t* s_r1 = one ? S.stage : nullptr;
     if (one)
         for (int i = tid; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
@@ -615,14 +622,14 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
             s_ovf_w[slot] = w;
             S.ovf_pos[slot] = pos;
         } else if (cnt > 4) {
-            store_ranked<WT_CAP>(src, S, w, pos, cnt, tc, s_r1, lc);
+            store_ranked<WT_CAP, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         } else if (cnt > 0) {
-            store_ranked<4>(src, S, w, pos, cnt, tc, s_r1, lc);
+            store_ranked<4, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         }
         __syncthreads();
         const uint32_t novf = (uint32_t)S.flag;
         for (uint32_t i = warp; i < novf; i += nwarps)
-            gather_rescan(src, S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
+            gather_rescan<kThr>(src, S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
         __syncthreads();
         run += piece;
     }
@@ -640,9 +647,20 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
             if (S.stage[i]) atomicAdd(&g[i], S.stage[i]);
     }
     mark_phase(cm.ctrl, 5);
-    if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return false;
+}
+
+// The gather phase, one grid barrier, and the decision every block takes
+// alike: candidates only if the list fit and each tensor kept at least k of
+// them with its k-th key inside the range of the relative digits.  Returns
+// false if the barrier gave up.
+__device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
+                                SelShared& S, uint64_t& my0, uint64_t& my1) {
+    gather_phase<false>(src, cm, S, my0, my1);
+    if (!grid_barrier(cm.bar, epoch, &cm.ctrl->status, &S.flag)) return false;
     mark_phase(cm.ctrl, 1);
 
+    const int T = src.T;
+    const int tid = threadIdx.x;
     const uint64_t total = (uint64_t)src.cand_start[T];
     const bool fits = total <= src.cap;
     uint32_t bad = 0;
@@ -651,11 +669,30 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
                src.rel_overflow(l);
     bad = block_sum(bad, S.red);
     src.dense = (src.force_dense || !fits || bad) ? 1 : 0;
-    if (c == 0 && tid == 0) {
+    if (blockIdx.x == 0 && tid == 0) {
         cm.ctrl->mode = src.dense;
         cm.ctrl->cand_total = total;
     }
     return true;
+}
+
+// Hard-threshold step ("Rethinking gradient sparsification as total error
+// minimization", abstract: Top-k with k set by a constant hard threshold):
+// the candidates of the streaming pass (key >= T0 = the threshold's key) are
+// the passing entries; the gather phase writes the first cap of them, in
+// index order, straight into the caller's output and zeroes their residual.
+// The last block writes the number that passed.
+__global__ void __launch_bounds__(SEL_THREADS)
+threshold_kernel(CompressSrc src, SelCommon cm, int64_t* out_count) {
+    __shared__ SelShared S;
+    mark_phase(cm.ctrl, 0);
+    uint64_t my0, my1;
+    gather_phase<true>(src, cm, S, my0, my1);
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+        *out_count = (int64_t)my1;
+        cm.ctrl->cand_total = my1;
+    }
+    mark_phase(cm.ctrl, 7);
 }
 
 // One pass over positions [a, b) of prefiltered tensor l (block-wide) once

@@ -22,6 +22,8 @@
 #include "kernels_compress.cuh"
 #include "kernels_merge.cuh"
 #include "kernels_select.cuh"
+#include "kernels_sparse.cuh"
+#include "kernels_merge_cluster.cuh"
 
 using namespace tke;
 
@@ -276,9 +278,14 @@ size_t groups_workspace(const std::vector<Group>& groups) {
 template <int TCAP>
 cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float* grad,
                          const float* resid, float lr, bool force_t0_zero, uint32_t kernels,
-                         cudaStream_t st) {
+                         cudaStream_t st, const uint32_t* fixed_T0 = nullptr) {
     SetupParams<TCAP> p;
     memset(&p, 0, sizeof(p));
+    if (fixed_T0) {
+        p.has_fixed_T0 = 1;
+        p.fixed_T0 = *fixed_T0;
+        force_t0_zero = true;          // no sampling
+    }
     const int T = (int)g.plans.size();
     p.grad = grad;
     p.resid = resid;
@@ -308,6 +315,57 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
     return launch_pdl(setup_kernel<TCAP>, ns + nz, SAMPLE_THREADS, st, p);
 }
 
+// The streaming pass of one group (after its setup kernel, with
+// programmatic serialisation); fills *sp for the select kernels.
+cudaError_t launch_stream(const Group& g, const CLayout& L, char* ws, const float* gg, float* rg,
+                          float lr, cudaStream_t st, const DevFacts& f, StreamParams* sp_out) {
+    StreamParams sp;
+    sp.grad = gg;
+    sp.resid = rg;
+    sp.lr = lr;
+    sp.T = (int)g.plans.size();
+    sp.N = g.N;
+    sp.num_wt = L.num_wt;
+    sp.meta = reinterpret_cast<const SegMeta*>(ws + L.meta);
+    sp.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+    sp.wt_count = reinterpret_cast<uint32_t*>(ws + L.wt_count);
+    sp.wt_off = reinterpret_cast<uint16_t*>(ws + L.wt_off);
+    *sp_out = sp;
+    const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
+    const int64_t warps_needed = L.num_wt;
+    const int g1 = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(warps_needed, K1_THREADS / 32),
+                                                               (int64_t)f.sms * f.k1_blocks));
+    trace_before(st, "stream_kernel");
+    cudaError_t e = vec ? launch_pdl(stream_kernel<true>, g1, K1_THREADS, st, sp)
+                        : launch_pdl(stream_kernel<false>, g1, K1_THREADS, st, sp);
+    trace_after(st);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e;
+}
+
+// Select-kernel view of a group's workspace (the compress defaults).
+CompressSrc make_src(const Group& g, const CLayout& L, char* ws, const StreamParams& sp,
+                     float* rg) {
+    CompressSrc src;
+    memset(&src, 0, sizeof(src));
+    src.resid = rg;
+    src.N = g.N;
+    src.T = (int)g.plans.size();
+    src.meta = sp.meta;
+    src.cand_start = reinterpret_cast<int64_t*>(ws + L.cand_start);
+    src.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
+    src.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
+    src.cap = (uint64_t)L.cap;
+    src.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+    src.num_wt = L.num_wt;
+    src.wt_count = sp.wt_count;
+    src.wt_off = sp.wt_off;
+    src.ent = reinterpret_cast<uint32_t*>(ws + L.ent);
+    src.ent_cnt = reinterpret_cast<uint32_t*>(ws + L.ent_cnt);
+    src.agg = reinterpret_cast<uint64_t*>(ws + L.agg);
+    return src;
+}
+
 int compress_group(const Group& g, const float* grad, float* resid, float lr, int32_t* out_idx,
                    float* out_val, char* ws, cudaStream_t st, const DevFacts& f, int flags) {
     const CLayout L = compress_layout(g.N, g.plans);
@@ -325,47 +383,13 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     if (e != cudaSuccess) return cuda_fail(e);
     if (g.N == 0) return TOPK_EF_OK;
 
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
     StreamParams sp;
-    sp.grad = gg;
-    sp.resid = rg;
-    sp.lr = lr;
-    sp.T = T;
-    sp.N = g.N;
-    sp.num_wt = L.num_wt;
-    sp.meta = reinterpret_cast<const SegMeta*>(ws + L.meta);
-    sp.ctrl = ctrl;
-    sp.wt_count = reinterpret_cast<uint32_t*>(ws + L.wt_count);
-    sp.wt_off = reinterpret_cast<uint16_t*>(ws + L.wt_off);
-    const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
-    const int64_t warps_needed = L.num_wt;
-    const int g1 = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(warps_needed, K1_THREADS / 32),
-                                                               (int64_t)f.sms * f.k1_blocks));
-    trace_before(st, "stream_kernel");
-    e = vec ? launch_pdl(stream_kernel<true>, g1, K1_THREADS, st, sp)
-            : launch_pdl(stream_kernel<false>, g1, K1_THREADS, st, sp);
-    trace_after(st);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp)) != cudaSuccess) return cuda_fail(e);
+    Ctrl* ctrl = sp.ctrl;
 
-    CompressSrc src;
-    memset(&src, 0, sizeof(src));
-    src.resid = rg;
-    src.N = g.N;
-    src.T = T;
-    src.meta = sp.meta;
-    src.cand_start = reinterpret_cast<int64_t*>(ws + L.cand_start);
-    src.cand_idx = reinterpret_cast<uint32_t*>(ws + L.cand_idx);
-    src.cand_val = reinterpret_cast<float*>(ws + L.cand_val);
-    src.cap = (uint64_t)L.cap;
-    src.hist = reinterpret_cast<uint32_t*>(ws + L.hist);
+    CompressSrc src = make_src(g, L, ws, sp, rg);
     src.out_idx = out_idx;
     src.out_val = out_val;
-    src.num_wt = L.num_wt;
-    src.wt_count = sp.wt_count;
-    src.wt_off = sp.wt_off;
-    src.ent = reinterpret_cast<uint32_t*>(ws + L.ent);
-    src.ent_cnt = reinterpret_cast<uint32_t*>(ws + L.ent_cnt);
-    src.agg = reinterpret_cast<uint64_t*>(ws + L.agg);
     src.force_dense = force_dense ? 1 : 0;
     src.dense = 0;
     SelCommon cm;
@@ -382,6 +406,108 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     trace_after(st);
     if (e != cudaSuccess) return cuda_fail(e);
     return TOPK_EF_OK;
+}
+
+// Hard-threshold step on one flat tensor: setup (fixed T0, no sampling),
+// the streaming pass, and the threshold kernel writing the output.
+int threshold_call(const float* grad, float* resid, int64_t n, float lr, uint32_t T0,
+                   int64_t max_out, int32_t* out_idx, float* out_val, int64_t* out_count,
+                   char* ws, cudaStream_t st, const DevFacts& f) {
+    Group g;
+    g.t0 = 0;
+    g.t1 = 1;
+    g.base = 0;
+    g.N = n;
+    TensorPlan t = plan_tensor(0, n, 0, 0);
+    t.cap = 0;
+    g.plans.push_back(t);
+    const CLayout L = compress_layout(n, g.plans);
+    const uint32_t kernels = n > 0 ? 3u : 1u;
+    trace_before(st, "setup_kernel");
+    cudaError_t e = launch_setup<TCAP_SMALL>(g, L, ws, grad, resid, lr, true, kernels, st, &T0);
+    trace_after(st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (n == 0) {
+        e = cudaMemsetAsync(out_count, 0, sizeof(int64_t), st);
+        return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
+    }
+    StreamParams sp;
+    if ((e = launch_stream(g, L, ws, grad, resid, lr, st, f, &sp)) != cudaSuccess)
+        return cuda_fail(e);
+    CompressSrc src = make_src(g, L, ws, sp, resid);
+    src.cand_idx = reinterpret_cast<uint32_t*>(out_idx);
+    src.cand_val = out_val;
+    src.cap = (uint64_t)std::min<int64_t>(max_out, n);
+    SelCommon cm;
+    cm.ctrl = sp.ctrl;
+    cm.bar = &sp.ctrl->bar;
+    cm.slots = reinterpret_cast<Slot*>(ws + L.slots);
+    const int G = std::min(SLOT_MAX, f.sms * std::min(1, f.selc_blocks));
+    void* args[] = {&src, &cm, &out_count};
+    trace_before(st, "threshold_kernel");
+    e = cudaLaunchCooperativeKernel((const void*)threshold_kernel, dim3(G), dim3(SEL_THREADS),
+                                    args, 0, st);
+    trace_after(st);
+    return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
+}
+
+size_t threshold_workspace(int64_t n) {
+    std::vector<TensorPlan> plans(1, plan_tensor(0, n, 0, 0));
+    plans[0].cap = 0;
+    return compress_layout(n, plans).total;
+}
+
+// The cluster merge kernel: shared memory attribute set once per device,
+// and at least one cluster of it must fit on the device.
+std::mutex g_mc_mu;
+int g_mc_state[64];             // 0 unknown, 1 usable, 2 not usable
+
+int merge_cluster_ready(bool* usable) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return TOPK_EF_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mc_mu);
+    if (g_mc_state[dev] == 0) {
+        e = cudaFuncSetAttribute(merge_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(McShared));
+        if (e != cudaSuccess) return cuda_fail(e);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(MC_CL);
+        cfg.blockDim = dim3(MC_THREADS);
+        cfg.dynamicSmemBytes = sizeof(McShared);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = MC_CL;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, merge_cluster_kernel, &cfg);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_mc_state[dev] = clusters > 0 ? 1 : 2;
+    }
+    *usable = g_mc_state[dev] == 1;
+    return TOPK_EF_OK;
+}
+
+cudaError_t launch_merge_cluster(int32_t np, cudaStream_t st, const MergeClusterParams& cp) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)np * MC_CL);
+    cfg.blockDim = dim3(MC_THREADS);
+    cfg.dynamicSmemBytes = sizeof(McShared);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = MC_CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, merge_cluster_kernel, cp);
 }
 
 bool bad_fp32_ptr(const void* p) { return ((uintptr_t)p & 3u) != 0; }
@@ -550,6 +676,141 @@ int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float
                             stream);
 }
 
+size_t topk_ef_threshold_workspace_bytes(int64_t n) {
+    if (n < 0 || n > MAX_N) return 0;
+    return threshold_workspace(n);
+}
+
+int topk_ef_threshold(const float* grad, float* residual, int64_t n, float lr, float threshold,
+                      int64_t max_out, int32_t* out_idx, float* out_val, int64_t* out_count,
+                      void* ws, size_t ws_bytes, void* stream) {
+    if (n < 0 || n > MAX_N || max_out < 0 || !out_count || !ws) return TOPK_EF_ERR_INVALID_ARG;
+    if (n > 0 && (!grad || !residual || bad_fp32_ptr(grad) || bad_fp32_ptr(residual)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (max_out > 0 && (!out_idx || !out_val || bad_fp32_ptr(out_idx) || bad_fp32_ptr(out_val)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (((uintptr_t)out_count % 8) != 0 || ((uintptr_t)ws % ALIGN) != 0)
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (ws_bytes < threshold_workspace(n)) return TOPK_EF_ERR_WORKSPACE;
+    DevFacts f;
+    int rc = device_facts(&f);
+    if (rc != TOPK_EF_OK) return rc;
+    // key of the threshold; never above 0x7F800001, so that the streaming
+    // pass's raw |bits| test and the key order agree (a NaN threshold passes
+    // exactly the NaNs)
+    uint32_t u;
+    memcpy(&u, &threshold, sizeof u);
+    uint32_t T0 = u & 0x7FFFFFFFu;
+    if (T0 > 0x7F800001u) T0 = 0x7F800001u;
+    return threshold_call(grad, residual, n, lr, T0, max_out, out_idx, out_val, out_count,
+                          (char*)ws, reinterpret_cast<cudaStream_t>(stream), f);
+}
+
+size_t gtopk_residual_return_workspace_bytes(void) { return align_up(sizeof(Ctrl)); }
+
+int gtopk_residual_return(const int32_t* sent_idx, const float* sent_val, int32_t P,
+                          int64_t k_sent, const int32_t* global_idx, int64_t k_global,
+                          float* residual, int64_t n, void* ws, size_t ws_bytes, void* stream) {
+    if (P < 1 || k_sent < 0 || k_global < 0 || n < 0 || n > MAX_N || k_sent > n || k_global > n)
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (!ws || ((uintptr_t)ws % ALIGN) != 0) return TOPK_EF_ERR_INVALID_ARG;
+    if (k_sent > 0 && (!sent_idx || !sent_val || !residual || bad_fp32_ptr(sent_idx) ||
+                       bad_fp32_ptr(sent_val) || bad_fp32_ptr(residual)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (k_global > 0 && (!global_idx || bad_fp32_ptr(global_idx))) return TOPK_EF_ERR_INVALID_ARG;
+    if (ws_bytes < gtopk_residual_return_workspace_bytes()) return TOPK_EF_ERR_WORKSPACE;
+    DevFacts f;
+    int rc = device_facts(&f);
+    if (rc != TOPK_EF_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(Ctrl), st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ReturnParams p;
+    p.sent_idx = sent_idx;
+    p.sent_val = sent_val;
+    p.k_sent = k_sent;
+    p.total = (int64_t)P * k_sent;
+    p.gidx = global_idx;
+    p.kg = k_global;
+    p.residual = residual;
+    p.n = n;
+    p.ctrl = reinterpret_cast<Ctrl*>(ws);
+    const int64_t work = std::max<int64_t>(p.total, k_global);
+    if (work == 0) return TOPK_EF_OK;
+    // one wave of resident blocks (grid-stride over the entries)
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, return_kernel, RET_THREADS,
+                                                           0)) != cudaSuccess)
+        return cuda_fail(e);
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div64(work, RET_THREADS), (int64_t)f.sms * std::max(1, per_sm)));
+    trace_before(st, "return_kernel");
+    return_kernel<<<grid, RET_THREADS, 0, st>>>(p);
+    trace_after(st);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
+}
+
+size_t topk_allgather_workspace_bytes(int32_t P, int64_t k_in, int64_t n) {
+    if (P < 1 || P > AG_MAX_P || k_in < 0 || n < 0 || n > MAX_N || k_in > n) return 0;
+    const int64_t nchunks = ceil_div64(n, AG_CHUNK);
+    return align_up(sizeof(Ctrl)) + align_up((size_t)(nchunks + 1) * P * sizeof(uint32_t));
+}
+
+int topk_allgather_sum(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k_in,
+                       int64_t n, float* out, void* ws, size_t ws_bytes, void* stream) {
+    const size_t need = topk_allgather_workspace_bytes(P, k_in, n);
+    if (need == 0 || !ws || ((uintptr_t)ws % ALIGN) != 0) return TOPK_EF_ERR_INVALID_ARG;
+    if (k_in > 0 && (!in_idx || !in_val || bad_fp32_ptr(in_idx) || bad_fp32_ptr(in_val)))
+        return TOPK_EF_ERR_INVALID_ARG;
+    if (n > 0 && (!out || bad_fp32_ptr(out))) return TOPK_EF_ERR_INVALID_ARG;
+    if (ws_bytes < need) return TOPK_EF_ERR_WORKSPACE;
+    DevFacts f;
+    int rc = device_facts(&f);
+    if (rc != TOPK_EF_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    AllGatherParams p;
+    p.idx = in_idx;
+    p.val = in_val;
+    p.P = P;
+    p.k_in = k_in;
+    p.n = n;
+    p.nchunks = ceil_div64(n, AG_CHUNK);
+    p.bound = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + align_up(sizeof(Ctrl)));
+    p.out = out;
+    p.ctrl = reinterpret_cast<Ctrl*>(ws);
+    const size_t bound_bytes = (size_t)(p.nchunks + 1) * P * sizeof(uint32_t);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(Ctrl), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.bound, 0xFF, bound_bytes, st);   // AG_UNSET
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (n == 0) return TOPK_EF_OK;
+    const int64_t total = (int64_t)P * k_in;
+    if (total > 0) {
+        const int gb = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(total, AG_THREADS),
+                                                                  (int64_t)f.sms * 8));
+        trace_before(st, "ag_bounds_kernel");
+        ag_bounds_kernel<<<gb, AG_THREADS, 0, st>>>(p);
+        trace_after(st);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    }
+    const size_t smem = (size_t)AG_WARPS * ag_warp_bytes(P);
+    if ((e = cudaFuncSetAttribute(ag_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+        return cuda_fail(e);
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ag_sum_kernel, AG_THREADS,
+                                                           smem)) != cudaSuccess)
+        return cuda_fail(e);
+    const int64_t want = ceil_div64(p.nchunks, AG_WARPS);
+    const int gs = (int)std::max<int64_t>(1, std::min<int64_t>(want,
+                                                              (int64_t)f.sms * std::max(1, per_sm)));
+    trace_before(st, "ag_sum_kernel");
+    ag_sum_kernel<<<gs, AG_THREADS, smem, st>>>(p);
+    trace_after(st);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
+}
+
 size_t gtopk_merge_workspace_bytes(int32_t P, int64_t k_in, int64_t k) {
     if (P < 1 || P > MAX_MERGE_P || k_in < 0 || k < 0) return 0;
     return merge_layout(P, k_in, k).total;
@@ -582,7 +843,13 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     uint32_t* m_idx = reinterpret_cast<uint32_t*>(w + L.m_idx);
     float* m_val = reinterpret_cast<float*>(w + L.m_val);
     const bool single = (P == 1 || k_in == 0);
-    const uint32_t kernels = single ? 2u : (uint32_t)(1 + 2 * L.rounds);
+    // one cluster kernel per round when every round's merged lists fit
+    bool cluster_path = !single;
+    for (int r = 0; r < L.rounds; ++r)
+        cluster_path = cluster_path && L.mcap[r] <= (int64_t)MC_CL * MC_Q;
+    if (cluster_path && (rc = merge_cluster_ready(&cluster_path)) != TOPK_EF_OK) return rc;
+    const uint32_t kernels =
+        single ? 2u : (uint32_t)(cluster_path ? 1 + L.rounds : 1 + 2 * L.rounds);
 
     MergeSetupParams sp;
     memset(&sp, 0, sizeof(sp));
@@ -648,6 +915,37 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
                                         dim3(SEL_THREADS), args, 0, st);
         trace_after(st);
         if (e != cudaSuccess) return cuda_fail(e);
+        return TOPK_EF_OK;
+    }
+
+    if (cluster_path) {
+        for (int r = 0; r < L.rounds; ++r) {
+            MergeClusterParams cp;
+            memset(&cp, 0, sizeof(cp));
+            cp.src_idx = r == 0 ? reinterpret_cast<const uint32_t*>(in_idx) : set_idx;
+            cp.src_val = r == 0 ? in_val : set_val;
+            cp.src_stride = r == 0 ? k_in : L.cap;
+            cp.sizes_in = r == 0 ? nullptr : sizes;
+            cp.size_const = (uint32_t)k_in;
+            cp.step = 1 << r;
+            cp.kmax = ms.kmax;
+            cp.dst_idx = set_idx;
+            cp.dst_val = set_val;
+            cp.dst_stride = L.cap;
+            cp.sizes_out = sizes;
+            cp.final_out = (r == L.rounds - 1) ? 1 : 0;
+            cp.out_idx = out_idx;
+            cp.out_val = out_val;
+            cp.out_count = out_count;
+            cp.out_k = k;
+            cp.bad_words = r == 0 ? bad : nullptr;
+            cp.n_bad = r == 0 ? (int32_t)L.vblocks : 0;
+            cp.ctrl = ctrl;
+            trace_before(st, "merge_cluster_kernel");
+            e = launch_merge_cluster(L.np[r], st, cp);
+            trace_after(st);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
         return TOPK_EF_OK;
     }
 

@@ -123,6 +123,39 @@ int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float
                             int64_t k, int32_t* out_idx, float* out_val,
                             void* stream);
 
+/* ------------------------------------------------------- hard threshold */
+
+/* Workspace bytes for topk_ef_threshold on n elements; 0 for invalid n. */
+size_t topk_ef_threshold_workspace_bytes(int64_t n);
+
+/*
+ * One error-feedback step of the hard-threshold sparsifier ("Rethinking
+ * gradient sparsification as total error minimization", abstract: the
+ * variant of Top-k whose k is set by a constant hard threshold, analysed
+ * under error feedback):
+ *     acc = fmaf(lr, grad, residual);
+ *     the entries with key(acc) >= key(threshold) pass (|acc| at least
+ *     |threshold|; NaN above +Inf, as in topk_ef_compress; a NaN threshold
+ *     passes only NaNs);
+ *     the first min(count, max_out) passing entries in ascending index order
+ *     are sent; the others stay in memory.
+ *   grad, residual, n, lr  as in topk_ef_compress
+ *   threshold  compared by magnitude (its sign is ignored)
+ *   max_out    >= 0: capacity of out_idx / out_val
+ *   out_idx    device, int32[max_out]: ascending indices of the sent entries;
+ *              slots from min(count, max_out) on are not written
+ *   out_val    device, fp32[max_out]: acc at those indices
+ *   out_count  device, int64 (8-byte aligned): count, the number of entries
+ *              that passed (may exceed max_out)
+ *   ws         device workspace of >= topk_ef_threshold_workspace_bytes(n)
+ * Errors: TOPK_EF_ERR_INVALID_ARG (n out of range, max_out < 0, null or
+ * misaligned pointers), TOPK_EF_ERR_WORKSPACE, TOPK_EF_ERR_CUDA.
+ */
+int topk_ef_threshold(const float* grad, float* residual, int64_t n, float lr,
+                      float threshold, int64_t max_out, int32_t* out_idx,
+                      float* out_val, int64_t* out_count, void* ws,
+                      size_t ws_bytes, void* stream);
+
 /* Workspace bytes for topk_ef_compress_batched with the same (offsets, k, T).
    offsets and k are host arrays.  Returns 0 for invalid arguments. */
 size_t topk_ef_batched_workspace_bytes(const int64_t* offsets,
@@ -178,6 +211,61 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P,
                 void* stream);
 
 /* ---------------------------------------------------------------- status */
+
+/* ------------------------------------------- after the gTop-k merge */
+
+/* Workspace bytes for gtopk_residual_return (a status block). */
+size_t gtopk_residual_return_workspace_bytes(void);
+
+/*
+ * Residual return after gTop-k: only the global set updates the model ("A
+ * Distributed Synchronous SGD Algorithm with Global Top-k Sparsification
+ * for Low Bandwidth Networks", ABSTRACT), so each worker puts back into its
+ * memory the values it sent whose index is not in the global set (error
+ * feedback: what is not transmitted accumulates locally, "The Convergence of
+ * Sparsified Gradient Methods", abstract):
+ *     for every worker p and sent (i, v) with i not in global_idx:
+ *         residual[p][i] = residual[p][i] + v          (one fp32 add)
+ *   sent_idx    device, int32[P][k_sent], each row strictly ascending in [0, n)
+ *               (the sets the workers sent, as given to gtopk_merge)
+ *   sent_val    device, fp32[P][k_sent]
+ *   global_idx  device, int32[k_global], strictly ascending in [0, n) (the
+ *               first out_count indices gtopk_merge returned)
+ *   residual    device, fp32[P][n], row p is worker p's memory
+ *   ws          device workspace of >= gtopk_residual_return_workspace_bytes()
+ * Malformed rows or global list: TOPK_EF_ERR_BAD_INPUT through
+ * topk_ef_last_device_status(ws); no memory outside residual is written.
+ * Errors: TOPK_EF_ERR_INVALID_ARG (P < 1, sizes out of range, null or
+ * misaligned pointers), TOPK_EF_ERR_WORKSPACE, TOPK_EF_ERR_CUDA.
+ */
+int gtopk_residual_return(const int32_t* sent_idx, const float* sent_val,
+                          int32_t P, int64_t k_sent, const int32_t* global_idx,
+                          int64_t k_global, float* residual, int64_t n,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes for topk_allgather_sum; 0 for invalid sizes
+   (1 <= P <= 256, 0 <= k_in <= n <= 2^31 - 1). */
+size_t topk_allgather_workspace_bytes(int32_t P, int64_t k_in, int64_t n);
+
+/*
+ * Top-k aggregation by AllGather, the O(kP) method the gTop-k review
+ * measures its merge against ("A Distributed Synchronous SGD Algorithm with
+ * Global Top-k Sparsification for Low Bandwidth Networks", ABSTRACT: current
+ * methods use AllGather to accumulate the sparse gradients), on one GPU:
+ * every worker's set is gathered and summed into a dense gradient in rank
+ * order,
+ *     out[i] = +0.0f;  for p = 0..P-1, for (i, v) in set p: out[i] += v
+ * (one fp32 add each, in that order).
+ *   in_idx   device, int32[P][k_in], rows strictly ascending in [0, n)
+ *   in_val   device, fp32[P][k_in]
+ *   out      device, fp32[n], written in full
+ *   ws       device workspace of >= topk_allgather_workspace_bytes(P, k_in, n)
+ * Malformed rows: TOPK_EF_ERR_BAD_INPUT through topk_ef_last_device_status;
+ * no memory outside out is written.
+ */
+int topk_allgather_sum(const int32_t* in_idx, const float* in_val, int32_t P,
+                       int64_t k_in, int64_t n, float* out, void* ws,
+                       size_t ws_bytes, void* stream);
 
 /* Synchronises `stream` and returns the device-side status of the last call
    that used `ws`: TOPK_EF_OK, TOPK_EF_ERR_DEVICE_TIMEOUT,

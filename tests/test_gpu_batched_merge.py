@@ -131,3 +131,21 @@ def test_merge_bad_input_flagged():
     good = np.array([[1, 3, 5], [0, 2, 4]], np.int32)
     ef.gtopk_merge(to_dev(good), to_dev(val), 3, 10, ws=ws)
     assert ef.topk_ef_last_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("P,k_in,k,n,cluster", [
+    (32, 25_557, 25_557, datagen.RESNET50_N, True),    # one cluster kernel per round
+    (4, 40_000, 40_000, 2_000_000, False),             # merged lists too long: merge + select
+    (32, 8_000, 40_000, 1_000_000, False),             # sets grow past the cluster size
+    (16, 30_000, 30_000, 500_000, True),
+])
+def test_merge_paths(P, k_in, k, n, cluster):
+    """Both round implementations: the cluster kernel (merge, select and
+    emission of a pair in one thread-block cluster) and the merge kernel +
+    grid-wide select; the launch count tells which one ran."""
+    idx, val = datagen.gtopk_sets(P=P, k=k_in, n=n, step=7)
+    ws = _mws(P, k_in, k)
+    run_merge(idx, val, k, n, ws=ws)
+    rounds = (P - 1).bit_length()
+    kernels = ef.topk_ef_path_info(ws)["kernels"]
+    assert kernels == (1 + rounds if cluster else 1 + 2 * rounds), kernels
