@@ -51,7 +51,7 @@ L2_BYTES = 126 << 20       # B200 L2; step inputs above this run back to back
 TRACE_EVERY = 8            # timed region: events around every 8th dominant launch
 LR = np.float32(0.1)
 POOL = 4          # distinct gradients cycled through the steps
-KERNEL_SOURCES = ["error_feedback_b200/csrc/kernels_compress.cuh",
+KERNEL_SOURCES = ["error_feedback_b200/csrc/kernels_stream.cuh",
                   "error_feedback_b200/csrc/common.cuh"]
 
 

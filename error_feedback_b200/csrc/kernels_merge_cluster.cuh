@@ -2,13 +2,23 @@
 // with Global Top-k Sparsification for Low Bandwidth Networks", ABSTRACT and
 // method section: worker i absorbs worker i + 2^r and keeps the top k of the
 // union, values at a common index added once).  Each pair of the round is
-// one thread-block cluster of MC_CL CTAs: CTA c of the cluster merges its
-// share of the merged list (merge path) into registers, the radix digits of
-// the k-th key are summed over the cluster through distributed shared memory
-// (cluster barriers, no grid barrier), and every CTA writes its share of the
-// top k in index order.  Used when a round's merged lists fit
-// (MC_CL * MC_Q positions per pair); larger rounds take the merge + select
-// kernels.
+// one thread-block cluster of CL CTAs:
+//   1. CTA c merges its share of the pair's merged list (merge path) into
+//      registers and builds the histogram of the first radix digit (key
+//      bits 30..20);
+//   2. the digit histograms are summed over the cluster through distributed
+//      shared memory, which gives the bin b1 of the k-th key;
+//   3. every CTA lists its entries in bin b1 (with its rank in the cluster)
+//      and counts those above it; every CTA then gathers all the lists and
+//      finds, locally, the k-th key T, the tie quota q and its own output
+//      offset (the counts above b1 of the CTAs before it plus their listed
+//      entries above / equal to T);
+//   4. every CTA writes its share of the top k in index order.
+// Three cluster barriers, no grid barrier.  A bin b1 with more entries than
+// the gather space resolves the remaining digits by two more summed
+// histogram passes and exchanges exact counts instead.  Used when a round's
+// merged lists fit (CL * QMAX positions per pair); larger rounds take the
+// merge + select kernels.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -20,10 +30,16 @@ namespace tke {
 
 namespace cg = cooperative_groups;
 
-constexpr int MC_CL = 8;                        // CTAs per pair
 constexpr int MC_THREADS = 512;
-constexpr int MC_PT = 16;                       // merged positions per thread at most
-constexpr int MC_Q = MC_THREADS * MC_PT;        // merged positions per CTA at most
+constexpr int64_t MC_PAIR_MAX = 65536;          // merged positions per pair
+
+template <int CL>
+struct McCfg {
+    static constexpr int PT = (int)(MC_PAIR_MAX / CL / MC_THREADS);   // positions per thread
+    static constexpr int QMAX = PT * MC_THREADS;                      // positions per CTA
+    static constexpr int STAGE = 4 * (QMAX + 1);                      // staging words
+    static constexpr int GCAP = STAGE - QMAX - 4;                     // gathered list capacity
+};
 
 struct MergeClusterParams {
     const uint32_t* src_idx;     // sets of this round, row stride src_stride
@@ -47,41 +63,81 @@ struct MergeClusterParams {
     Ctrl* ctrl;
 };
 
-// Shared memory of one CTA.
-struct McShared {
+// Fixed part of a CTA's shared memory; the staging words follow it.
+struct McFixed {
     uint32_t h1[D1_BINS], h2[D2_BINS], h3[D3_BINS];   // this CTA's digit histograms
-    uint32_t tot[D1_BINS];                            // cluster sums
+    uint32_t tot[D1_BINS];                            // cluster sums / local histograms
     uint64_t scan[33];
     uint32_t red[33];
     int64_t part[2];
-    uint32_t live, gt, eq;
+    uint32_t live, above, nlist, gt, eq, pg, pe;
+    uint32_t loff[17];                                // list offsets by cluster rank
+    uint32_t E, pre_above;
     FindResult fr;
-    uint32_t sAi[MC_Q + 1], sBi[MC_Q + 1];
-    float sAv[MC_Q + 1], sBv[MC_Q + 1];
 };
+
+template <int CL>
+constexpr size_t mc_smem_bytes() {
+    return (sizeof(McFixed) + 15) / 16 * 16 + (size_t)McCfg<CL>::STAGE * 4;
+}
 
 // Sum of histogram `h` (nb bins) over the cluster into S.tot, then the bin of
 // the rem-th largest; every CTA computes the same.
-__device__ __forceinline__ void cluster_find(cg::cluster_group& cl, McShared& S, uint32_t* h,
-                                             int nb, uint32_t rem) {
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+// All remote loads of a thread are issued before the first is summed (NB is
+// a multiple of MC_THREADS).
+template <int CL, int NB>
+__device__ __forceinline__ void cluster_find(cg::cluster_group& cl, McFixed& S, uint32_t* h,
+                                             uint32_t rem) {
+    constexpr int PER = NB / MC_THREADS;
+    uint32_t v[PER][CL];
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+#pragma unroll
+        for (int r = 0; r < CL; ++r) v[j][r] = *cl.map_shared_rank(h + threadIdx.x + j * MC_THREADS, r);
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
         uint32_t s = 0;
 #pragma unroll
-        for (int r = 0; r < MC_CL; ++r) s += *cl.map_shared_rank(h + i, r);
-        S.tot[i] = s;
+        for (int r = 0; r < CL; ++r) s += v[j][r];
+        S.tot[threadIdx.x + j * MC_THREADS] = s;
+    }
+    __syncthreads();
+    block_find_bin(S.tot, NB, rem, S.red, &S.fr);
+}
+
+// Local histogram of `nb` bins over the gathered list (entries whose `sel`
+// holds), then the bin of the rem-th largest (result in S.fr).
+template <class Sel, class Bin>
+__device__ __forceinline__ void list_find(McFixed& S, const uint32_t* list, uint32_t E, int nb,
+                                          uint32_t rem, Sel sel, Bin bin) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) S.tot[i] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < E; i += blockDim.x) {
+        const uint32_t v = list[i];
+        if (sel(v)) atomicAdd(&S.tot[bin(v)], 1u);
     }
     __syncthreads();
     block_find_bin(S.tot, nb, rem, S.red, &S.fr);
 }
 
-__global__ void __launch_bounds__(MC_THREADS, 1)
+template <int CL>
+__global__ void __launch_bounds__(MC_THREADS, (CL >= 16 ? 2 : 1))
 merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
+    using C = McCfg<CL>;
+    constexpr int PT = C::PT;
+    constexpr int QMAX = C::QMAX;
     extern __shared__ __align__(16) unsigned char mc_smem[];
-    McShared& S = *reinterpret_cast<McShared*>(mc_smem);
+    McFixed& S = *reinterpret_cast<McFixed*>(mc_smem);
+    uint32_t* stage = reinterpret_cast<uint32_t*>(mc_smem + (sizeof(McFixed) + 15) / 16 * 16);
+    uint32_t* sAi = stage;
+    uint32_t* sBi = stage + (QMAX + 1);
+    float* sAv = reinterpret_cast<float*>(stage + 2 * (QMAX + 1));
+    float* sBv = reinterpret_cast<float*>(stage + 3 * (QMAX + 1));
     cg::cluster_group cl = cg::this_cluster();
     const int tid = threadIdx.x;
     const int cr = (int)cl.block_rank();
-    const int pair = blockIdx.x / MC_CL;
+    const int pair = blockIdx.x / CL;
     // the previous round's sets and sizes (programmatic serialisation)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const bool stamp = blockIdx.x == 0 && tid == 0;     // diagnostics: CTA 0's phases
@@ -102,7 +158,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     const float* Av = p.src_val + left * p.src_stride;
     const float* Bv = p.src_val + right * p.src_stride;
     const int64_t ab = a + b;
-    const int64_t Q = (ab + MC_CL - 1) / MC_CL;          // <= MC_Q (host check)
+    const int64_t Q = (ab + CL - 1) / CL;                // <= QMAX (host check)
     const int64_t d0 = min((int64_t)cr * Q, ab);
     const int64_t d1 = min(d0 + Q, ab);
     if (tid < 64) {
@@ -117,64 +173,85 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     if (stamp) p.ctrl->t_phase[1] = global_ns();
     const int64_t i0 = S.part[0], i1 = max(S.part[1], i0);
     const int64_t j0 = d0 - i0, j1 = max(d1 - S.part[1], j0);
-    const int la = (int)min(i1 - i0, (int64_t)MC_Q);
-    const int lb = (int)min(j1 - j0, (int64_t)MC_Q);
-    // sA[x] = A[i0 - 1 + x] for x in [0, la]; sB[y] = B[j0 + y] for y in [0, lb]
-    for (int x = tid; x <= la; x += blockDim.x) {
-        const int64_t gi = i0 - 1 + x;
-        const bool in = gi >= 0 && gi < a;
-        S.sAi[x] = in ? Ai[gi] : DEAD;
-        S.sAv[x] = in ? Av[gi] : 0.f;
-    }
-    for (int y = tid; y <= lb; y += blockDim.x) {
-        const int64_t gj = j0 + y;
-        const bool in = gj < b;
-        S.sBi[y] = in ? Bi[gj] : DEAD;
-        S.sBv[y] = in ? Bv[gj] : 0.f;
+    const int la = (int)min(i1 - i0, (int64_t)QMAX);
+    const int lb = (int)min(j1 - j0, (int64_t)QMAX);
+    // sA[x] = A[i0 - 1 + x] for x in [0, la]; sB[y] = B[j0 + y] for y in [0, lb];
+    // all loads of a thread are issued before its stores
+    {
+        uint32_t ri[PT + 1];
+        float rv[PT + 1];
+#pragma unroll
+        for (int u = 0; u <= PT; ++u) {
+            const int x = tid + u * MC_THREADS;
+            const int64_t gi = i0 - 1 + x;
+            const bool in = x <= la && gi >= 0 && gi < a;
+            ri[u] = in ? Ai[gi] : DEAD;
+            rv[u] = in ? Av[gi] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u <= PT; ++u) {
+            const int x = tid + u * MC_THREADS;
+            if (x <= la) {
+                sAi[x] = ri[u];
+                sAv[x] = rv[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u <= PT; ++u) {
+            const int y = tid + u * MC_THREADS;
+            const int64_t gj = j0 + y;
+            const bool in = y <= lb && gj < b;
+            ri[u] = in ? Bi[gj] : DEAD;
+            rv[u] = in ? Bv[gj] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u <= PT; ++u) {
+            const int y = tid + u * MC_THREADS;
+            if (y <= lb) {
+                sBi[y] = ri[u];
+                sBv[y] = rv[u];
+            }
+        }
     }
     __syncthreads();
     if (stamp) p.ctrl->t_phase[2] = global_ns();
 
-    // merge this thread's positions [dl, dl + MC_PT) of the CTA's span
+    // merge this thread's positions [dl, dl + pt) of the CTA's span
     const int span = (int)(d1 - d0);
-    const int pt = (span + MC_THREADS - 1) / MC_THREADS;  // positions per thread
+    const int pt = (span + MC_THREADS - 1) / MC_THREADS;
     const int dl = tid * pt;
-    uint32_t mi[MC_PT];
-    float mv[MC_PT];
+    uint32_t mi[PT];
+    float mv[PT];
     uint32_t live = 0;
     {
         int ia = 0, ib = 0;
         if (dl < span) {
-            ia = local_merge_path(S.sAi + 1, la, S.sBi, lb, dl);
+            ia = local_merge_path(sAi + 1, la, sBi, lb, dl);
             ib = dl - ia;
         }
 #pragma unroll
-        for (int u = 0; u < MC_PT; ++u) {
+        for (int u = 0; u < PT; ++u) {
             uint32_t oi = DEAD;
             float ov = 0.f;
             const int pos = dl + u;
             if (u < pt && pos < span) {
                 const int64_t d = d0 + pos;
-                const bool takeA = ia < la && (ib >= lb || S.sAi[1 + ia] <= S.sBi[ib]);
+                const bool takeA = ia < la && (ib >= lb || sAi[1 + ia] <= sBi[ib]);
                 if (takeA) {
-                    oi = S.sAi[1 + ia];
-                    ov = S.sAv[1 + ia];
+                    oi = sAi[1 + ia];
+                    ov = sAv[1 + ia];
                     // partner: the next B element, B[d - i] with i = i0 + ia
-                    const int64_t jB = d - (i0 + ia);
-                    if (jB < b) {
-                        const int64_t y = jB - j0;
-                        if (y >= 0 && y <= lb && S.sBi[y] == oi) ov = __fadd_rn(ov, S.sBv[y]);
-                    }
+                    const int64_t y = d - (i0 + ia) - j0;
+                    if (d - (i0 + ia) < b && y >= 0 && y <= lb && sBi[y] == oi)
+                        ov = __fadd_rn(ov, sBv[y]);
                     ++ia;
                 } else {
-                    oi = ib < lb ? S.sBi[ib] : DEAD;
-                    ov = ib < lb ? S.sBv[ib] : 0.f;
+                    oi = ib < lb ? sBi[ib] : DEAD;
+                    ov = ib < lb ? sBv[ib] : 0.f;
                     // the previous A element, A[iA - 1] with iA = d - j
                     const int64_t iA = d - (j0 + ib);
-                    if (iA > 0) {
-                        const int64_t x = iA - i0;       // sA[x] = A[iA - 1]
-                        if (x >= 0 && x <= la && S.sAi[x] == oi) oi = DEAD;
-                    }
+                    const int64_t x = iA - i0;           // sA[x] = A[iA - 1]
+                    if (iA > 0 && x >= 0 && x <= la && sAi[x] == oi) oi = DEAD;
                     ++ib;
                 }
             }
@@ -189,55 +266,179 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     live = block_sum(live, S.red);
     if (tid == 0) S.live = live;
     if (stamp) p.ctrl->t_phase[3] = global_ns();
-    cl.sync();                                           // h1 and live of every CTA
+    cl.sync();                                           // [1] h1 and live of every CTA
     if (stamp) p.ctrl->t_phase[4] = global_ns();
 
     uint32_t live_tot = 0;
 #pragma unroll
-    for (int r = 0; r < MC_CL; ++r) live_tot += *cl.map_shared_rank(&S.live, r);
+    for (int r = 0; r < CL; ++r) live_tot += *cl.map_shared_rank(&S.live, r);
     const uint32_t kp = live_tot < p.kmax ? live_tot : p.kmax;
-    uint32_t T = NO_KEY, q = 0;
-    uint32_t rem = kp, b1 = 0, b2 = 0;
+    uint32_t b1 = 0, rem = kp;
     bool ok = kp > 0;
-    if (ok) {
-        cluster_find(cl, S, S.h1, D1_BINS, rem);
+    if (kp > 0) {
+        cluster_find<CL, D1_BINS>(cl, S, S.h1, rem);
         ok = S.fr.ok;
         b1 = S.fr.bin;
         rem -= S.fr.above;
-#pragma unroll
-        for (int u = 0; u < MC_PT; ++u)
-            if (mi[u] != DEAD && (key_of(mv[u]) >> 20) == b1)
-                atomicAdd(&S.h2[(key_of(mv[u]) >> 10) & (D2_BINS - 1)], 1u);
     }
-    cl.sync();                                           // h2
-    if (kp > 0) {
-        cluster_find(cl, S, S.h2, D2_BINS, rem);
-        ok = ok && S.fr.ok;
-        b2 = S.fr.bin;
-        rem -= S.fr.above;
-        const uint32_t pre = (b1 << D2_BITS) | b2;
+    // this CTA's entries in bin b1 (low 20 key bits, in the staging space,
+    // which the merge no longer needs) and its count above b1
+    uint32_t* mylist = stage;                           // [QMAX]
+    uint32_t* glist = stage + QMAX + 4;                 // [GCAP]
+    {
+        uint32_t nin = 0, nab = 0;
 #pragma unroll
-        for (int u = 0; u < MC_PT; ++u)
-            if (mi[u] != DEAD && (key_of(mv[u]) >> 10) == pre)
-                atomicAdd(&S.h3[key_of(mv[u]) & (D3_BINS - 1)], 1u);
-    }
-    cl.sync();                                           // h3
-    if (kp > 0) {
-        cluster_find(cl, S, S.h3, D3_BINS, rem);
-        ok = ok && S.fr.ok;
-        T = (b1 << 20) | (b2 << 10) | S.fr.bin;
-        q = rem - S.fr.above;
-        if (!ok) {
-            if (tid == 0) atomicOr(&p.ctrl->status, ST_INCONSISTENT);
-            T = NO_KEY;
-            q = 0;
+        for (int u = 0; u < PT; ++u) {
+            if (mi[u] == DEAD || kp == 0) continue;
+            const uint32_t d = key_of(mv[u]) >> 20;
+            nin += d == b1;
+            nab += d > b1;
+        }
+        __syncthreads();                                 // staging reads are done
+        uint32_t tin;
+        uint32_t at = block_excl_scan(nin, S.red, &tin);
+#pragma unroll
+        for (int u = 0; u < PT; ++u) {
+            if (mi[u] == DEAD || kp == 0) continue;
+            const uint32_t key = key_of(mv[u]);
+            if ((key >> 20) == b1) mylist[at++] = ((uint32_t)cr << 20) | (key & 0xFFFFFu);
+        }
+        nab = block_sum(nab, S.red);
+        if (tid == 0) {
+            S.nlist = tin;
+            S.above = nab;
         }
     }
+    cl.sync();                                           // [2] every CTA's list and count
     if (stamp) p.ctrl->t_phase[5] = global_ns();
-    // this thread's (key > T, key == T) counts, then the CTA's
+
+    // list lengths and counts above b1 of all CTAs (lane r reads rank r)
+    if (tid < 32) {
+        const uint32_t lane = lane_id();
+        uint32_t nr = 0, ar = 0;
+        if (lane < (uint32_t)CL) {
+            nr = *cl.map_shared_rank(&S.nlist, (int)lane);
+            ar = *cl.map_shared_rank(&S.above, (int)lane);
+        }
+        const uint32_t incl = warp_incl_scan(nr);
+        if (lane < (uint32_t)CL) S.loff[lane] = incl - nr;
+        if (lane == (uint32_t)CL - 1) S.loff[CL] = incl;
+        const uint32_t pa = warp_sum((int)lane < cr ? ar : 0u);
+        const uint32_t all = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (lane == 0) {
+            S.E = all;
+            S.pre_above = pa;
+        }
+    }
+    __syncthreads();
+    const uint32_t E = S.E, pre_above = S.pre_above;
+    uint32_t T = NO_KEY, q = 0, pg = 0, pe = 0;
+    const bool gathered = E <= (uint32_t)C::GCAP;       // the same in every CTA
+    if (gathered) {
+        // all lists, in cluster rank order: batches of GU independent
+        // remote loads per thread
+        constexpr int GU = 8;
+        for (uint32_t g0 = tid; g0 < E; g0 += GU * blockDim.x) {
+            uint32_t v[GU];
+#pragma unroll
+            for (int u = 0; u < GU; ++u) {
+                const uint32_t g = g0 + u * blockDim.x;
+                v[u] = 0;
+                if (g < E) {
+                    int r = 0;
+#pragma unroll
+                    for (int st = CL / 2; st >= 1; st >>= 1)
+                        if (r + st < CL && S.loff[r + st] <= g) r += st;
+                    v[u] = *cl.map_shared_rank(mylist + (g - S.loff[r]), r);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < GU; ++u)
+                if (g0 + u * blockDim.x < E) glist[g0 + u * blockDim.x] = v[u];
+        }
+        if (kp > 0 && ok) {
+            // bits 19..10, then 9..0 of the k-th key inside bin b1
+            list_find(S, glist, E, 1024, rem, [](uint32_t) { return true; },
+                      [](uint32_t v) { return (v >> 10) & 1023u; });
+            const uint32_t bA = S.fr.bin;
+            const uint32_t remA = rem - S.fr.above;
+            ok = S.fr.ok;
+            list_find(S, glist, E, 1024, remA,
+                      [bA](uint32_t v) { return ((v >> 10) & 1023u) == bA; },
+                      [](uint32_t v) { return v & 1023u; });
+            ok = ok && S.fr.ok;
+            const uint32_t t = (bA << 10) | S.fr.bin;
+            q = remA - S.fr.above;
+            T = ok ? (b1 << 20) | t : NO_KEY;
+            // entries of earlier CTAs in bin b1: above T, equal to T
+            uint32_t g = 0, e = 0;
+            for (uint32_t i = tid; i < E; i += blockDim.x) {
+                const uint32_t v = glist[i];
+                if ((int)(v >> 20) < cr) {
+                    g += (v & 0xFFFFFu) > t;
+                    e += (v & 0xFFFFFu) == t;
+                }
+            }
+            g = block_sum(g, S.red);
+            e = block_sum(e, S.red);
+            pg = pre_above + g;
+            pe = e;
+        }
+    } else {
+        // crowded bin: two more summed digit passes, then exact counts
+        if (kp > 0) {
+#pragma unroll
+            for (int u = 0; u < PT; ++u)
+                if (mi[u] != DEAD && (key_of(mv[u]) >> 20) == b1)
+                    atomicAdd(&S.h2[(key_of(mv[u]) >> 10) & (D2_BINS - 1)], 1u);
+        }
+        cl.sync();
+        uint32_t b2 = 0;
+        if (kp > 0) {
+            cluster_find<CL, D2_BINS>(cl, S, S.h2, rem);
+            ok = ok && S.fr.ok;
+            b2 = S.fr.bin;
+            rem -= S.fr.above;
+            const uint32_t pre = (b1 << D2_BITS) | b2;
+#pragma unroll
+            for (int u = 0; u < PT; ++u)
+                if (mi[u] != DEAD && (key_of(mv[u]) >> 10) == pre)
+                    atomicAdd(&S.h3[key_of(mv[u]) & (D3_BINS - 1)], 1u);
+        }
+        cl.sync();
+        if (kp > 0) {
+            cluster_find<CL, D3_BINS>(cl, S, S.h3, rem);
+            ok = ok && S.fr.ok;
+            q = rem - S.fr.above;
+            T = ok ? (b1 << 20) | (b2 << 10) | S.fr.bin : NO_KEY;
+        }
+        uint32_t g = 0, e = 0;
+#pragma unroll
+        for (int u = 0; u < PT; ++u) {
+            if (mi[u] == DEAD || T == NO_KEY) continue;
+            const uint32_t key = key_of(mv[u]);
+            g += key > T;
+            e += key == T;
+        }
+        g = block_sum(g, S.red);
+        e = block_sum(e, S.red);
+        if (tid == 0) {
+            S.gt = g;
+            S.eq = e;
+        }
+        cl.sync();
+        for (int r = 0; r < cr; ++r) {
+            pg += *cl.map_shared_rank(&S.gt, r);
+            pe += *cl.map_shared_rank(&S.eq, r);
+        }
+    }
+    if (kp > 0 && T == NO_KEY && tid == 0) atomicOr(&p.ctrl->status, ST_INCONSISTENT);
+    if (stamp) p.ctrl->t_phase[6] = global_ns();
+
+    // emission in index order: rank = #gt + min(#eq, q) before the entry
     uint32_t g = 0, e = 0;
 #pragma unroll
-    for (int u = 0; u < MC_PT; ++u) {
+    for (int u = 0; u < PT; ++u) {
         if (mi[u] == DEAD || T == NO_KEY) continue;
         const uint32_t key = key_of(mv[u]);
         g += key > T;
@@ -245,24 +446,12 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     }
     uint64_t tot_ge;
     const uint64_t ex = block_excl_scan(((uint64_t)g << 32) | e, S.scan, &tot_ge);
-    if (tid == 0) {
-        S.gt = (uint32_t)(tot_ge >> 32);
-        S.eq = (uint32_t)(tot_ge & 0xFFFFFFFFu);
-    }
-    cl.sync();                                           // every CTA's counts
-    if (stamp) p.ctrl->t_phase[6] = global_ns();
-    uint32_t pg = 0, pe = 0;
-    for (int r = 0; r < cr; ++r) {
-        pg += *cl.map_shared_rank(&S.gt, r);
-        pe += *cl.map_shared_rank(&S.eq, r);
-    }
-    // emission in index order: rank = #gt + min(#eq, q) before the entry
     if (T != NO_KEY) {
         uint32_t rg = pg + (uint32_t)(ex >> 32), re = pe + (uint32_t)(ex & 0xFFFFFFFFu);
         uint32_t* di = p.dst_idx + left * p.dst_stride;
         float* dv = p.dst_val + left * p.dst_stride;
 #pragma unroll
-        for (int u = 0; u < MC_PT; ++u) {
+        for (int u = 0; u < PT; ++u) {
             if (mi[u] == DEAD) continue;
             const uint32_t key = key_of(mv[u]);
             uint32_t rank = 0xFFFFFFFFu;
@@ -288,7 +477,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         // result length and the padding of the caller's arrays
         if (cr == 0 && tid == 0) *p.out_count = (int32_t)kp;
         for (int64_t i = (int64_t)kp + (int64_t)cr * blockDim.x + tid; i < p.out_k;
-             i += (int64_t)MC_CL * blockDim.x) {
+             i += (int64_t)CL * blockDim.x) {
             p.out_idx[i] = -1;
             p.out_val[i] = 0.0f;
         }

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "kernels_compress.cuh"
+#include "kernels_stream.cuh"
 
 namespace tke {
 

@@ -1,0 +1,216 @@
+// The fused streaming pass of the compress step ("Sparsified SGD with
+// Memory" and "The Convergence of Sparsified Gradient Methods", abstracts in
+// the arxivdaily listing): acc = fmaf(lr, grad, residual) written back to the
+// residual, and the positions of the entries whose key reaches the
+// prefilter threshold T0 recorded per warp tile.  The only full sweep of a
+// step; everything it needs from the setup kernel is in SegMeta.
+#pragma once
+
+#include "common.cuh"
+#include "kernels_compress.cuh"
+
+namespace tke {
+
+struct StreamParams {
+    const float* grad;
+    float* resid;
+    float lr;
+    int32_t T;
+    int64_t N;
+    uint32_t num_wt;        // warp tiles of WT elements
+    const SegMeta* meta;
+    Ctrl* ctrl;
+    uint32_t* wt_count;     // [num_wt] candidates of each warp tile (exact)
+    uint16_t* wt_off;       // [num_wt][WT_CAP]: their offsets in the tile, unordered
+};
+
+// Tensor l with off[l] <= e < off[l+1] (empty tensors are skipped).
+__device__ __forceinline__ int seg_of(const int64_t* off, int T, int64_t e) {
+    int lo = 0, hi = T;   // answer in [0, T)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (off[mid] <= e) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// First l in [0, T] with off[l] >= e.
+__device__ __forceinline__ int lower_bound_off(const int64_t* off, int T, int64_t e) {
+    int lo = 0, hi = T + 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (off[mid] < e) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+struct StreamShared {
+    int64_t off[TCAP_LARGE + 1];
+    uint32_t T0[TCAP_LARGE];
+};
+
+// General warp tile: a partial last tile, a tile that spans tensors, or
+// unaligned inputs.  Computes acc, stores it, returns the candidate flags
+// (bit 4j + v for element base + 128 j + 4 lane + v).
+template <bool VEC>
+__device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, const StreamShared& S,
+                                                     int64_t base, int l_lo, int l_hi) {
+    const uint32_t lane = lane_id();
+    uint32_t flags = 0;
+    for (int j = 0; j < WT_VECS; ++j) {
+        const int64_t e = base + j * 128 + lane * 4;
+        float a[4];
+        if (VEC && e + 3 < p.N) {
+            const float4 gv = ld_stream(reinterpret_cast<const float4*>(p.grad + e));
+            const float4 rv = ld_stream(reinterpret_cast<const float4*>(p.resid + e));
+            a[0] = __fmaf_rn(p.lr, gv.x, rv.x);
+            a[1] = __fmaf_rn(p.lr, gv.y, rv.y);
+            a[2] = __fmaf_rn(p.lr, gv.z, rv.z);
+            a[3] = __fmaf_rn(p.lr, gv.w, rv.w);
+            st_stream(reinterpret_cast<float4*>(p.resid + e), make_float4(a[0], a[1], a[2], a[3]));
+        } else {
+            for (int v = 0; v < 4; ++v) {
+                a[v] = 0.f;
+                if (e + v < p.N) {
+                    a[v] = __fmaf_rn(p.lr, __ldcs(p.grad + e + v), __ldcs(p.resid + e + v));
+                    __stcs(p.resid + e + v, a[v]);
+                }
+            }
+        }
+        for (int v = 0; v < 4; ++v) {
+            if (e + v >= p.N) continue;
+            int l = l_lo;
+            while (l < l_hi && S.off[l + 1] <= e + v) ++l;
+            if (key_of(a[v]) >= S.T0[l]) flags |= 1u << (j * 4 + v);
+        }
+    }
+    return flags;
+}
+
+// Record the candidates of a warp tile: the exact count and, up to WT_CAP of
+// them, their offsets in the tile (lane-major, so not in index order; the
+// select kernel sorts each tile's few offsets and reads the values back from
+// the residual, which now holds acc).  Bit 4j + v of a lane's flags is offset
+// 128 j + 4 lane + v.
+__device__ __forceinline__ void stream_tile_stage(const StreamParams& p, uint32_t w, uint32_t flags) {
+    const uint32_t lane = lane_id();
+    const uint32_t pc = (uint32_t)__popc(flags);
+    const uint32_t incl = warp_incl_scan(pc);
+    if (lane == 31) p.wt_count[w] = incl;
+    uint32_t pos = incl - pc;
+    uint16_t* dst = p.wt_off + (size_t)w * WT_CAP;
+    while (flags && pos < (uint32_t)WT_CAP) {
+        const uint32_t b = (uint32_t)(__ffs(flags) - 1);
+        flags &= flags - 1;
+        dst[pos++] = (uint16_t)(128u * (b >> 2) + 4u * lane + (b & 3u));
+    }
+}
+
+__device__ __forceinline__ void stream_tile_record(const StreamParams& p, uint32_t w,
+                                                   uint32_t flags) {
+    if (__any_sync(0xFFFFFFFFu, flags != 0)) stream_tile_stage(p, w, flags);
+    else if (lane_id() == 0) p.wt_count[w] = 0;
+}
+
+// The fused streaming pass, the only full sweep of the step:
+//   acc = fmaf(lr, grad, residual) written back to residual;
+//   candidates (key >= T0 of the element's tensor) recorded per warp tile of
+//   1,024 elements: an exact count and the offsets of up to WT_CAP of them.
+// Each warp owns whole warp tiles, so warps never wait for one another; the
+// select kernel rebuilds the ordered candidate list from the records.  The loop
+// over full tiles of one tensor is kept small; everything else is out of line.
+template <bool VEC>
+__global__ void __launch_bounds__(K1_THREADS, 3)
+stream_kernel(const __grid_constant__ StreamParams p) {
+    __shared__ StreamShared S;
+    const int tid = threadIdx.x;
+    {
+        // While the setup kernel still runs (this grid is launched early),
+        // pull this warp's first warp tiles into L2: the reads do not depend
+        // on it, only the writes and the candidate test do.
+        const uint32_t warps = blockDim.x >> 5;
+        const uint32_t gw0 = blockIdx.x * warps + warp_id();
+        const uint32_t GW0 = gridDim.x * warps;
+        const uint32_t R0 = p.num_wt / GW0 >= 2 ? p.num_wt / GW0 - 1 : 0;
+        if (VEC && lane_id() == 0) {
+            for (uint32_t i = 0; i < STREAM_PREFETCH && i < R0; ++i) {
+                const int64_t base = (int64_t)(gw0 + i * GW0) * WT;
+                if (base + WT > p.N) break;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.grad + base),
+                             "r"((uint32_t)(WT * 4))
+                             : "memory");
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.resid + base),
+                             "r"((uint32_t)(WT * 4))
+                             : "memory");
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // setup_kernel's results
+    const uint32_t lane = lane_id();
+    const int T = p.T;
+    const bool flat = (T == 1);
+    for (int l = tid; l < T; l += blockDim.x) {
+        S.off[l] = p.meta[l].off;
+        S.T0[l] = p.meta[l].T0;
+    }
+    if (tid == 0) S.off[T] = p.N;
+    __syncthreads();
+
+    // Warp tiles are handed out statically for all but the last rounds, then
+    // by ticket, so that no warp is left with a whole extra round at the end.
+    const uint32_t warps = blockDim.x >> 5;
+    const uint32_t gw = blockIdx.x * warps + warp_id();
+    const uint32_t GW = gridDim.x * warps;
+    const uint32_t R = p.num_wt / GW >= 2 ? p.num_wt / GW - 1 : 0;   // static rounds
+    const float lr = p.lr;
+    uint32_t w;
+    if (R > 0) {
+        w = gw;
+    } else {
+        uint32_t t = 0;
+        if (lane == 0) t = atomicAdd(&p.ctrl->tile_ticket, 1u);
+        w = R * GW + __shfl_sync(0xFFFFFFFFu, t, 0);
+    }
+    for (uint32_t round = 0; w < p.num_wt; ++round) {
+        // next tile: static, or a ticket fetched now and read after this tile
+        uint32_t ticket = 0;
+        const bool stat_next = round + 1 < R;
+        if (!stat_next && lane == 0) ticket = atomicAdd(&p.ctrl->tile_ticket, 1u);
+        const int64_t base = (int64_t)w * WT;
+        const int64_t tend = min(base + (int64_t)WT, p.N);
+        const int l_lo = flat ? 0 : seg_of(S.off, T, base);
+        const int l_hi = flat ? 0 : seg_of(S.off, T, tend - 1);
+        if (VEC && l_lo == l_hi && tend - base == WT) {
+            // full warp tile inside one tensor: 128-bit loads, no bounds checks
+            const uint32_t T0 = S.T0[l_lo];
+            const float4* g4 = reinterpret_cast<const float4*>(p.grad + base) + lane;
+            float4* r4 = reinterpret_cast<float4*>(p.resid + base) + lane;
+            float4 gv[WT_VECS], rv[WT_VECS];
+#pragma unroll
+            for (int j = 0; j < WT_VECS; ++j) {
+                gv[j] = ld_stream(g4 + 32 * j);
+                rv[j] = ld_stream(r4 + 32 * j);
+            }
+            uint32_t flags = 0;
+#pragma unroll
+            for (int j = 0; j < WT_VECS; ++j) {
+                float4 a;
+                a.x = __fmaf_rn(lr, gv[j].x, rv[j].x);
+                a.y = __fmaf_rn(lr, gv[j].y, rv[j].y);
+                a.z = __fmaf_rn(lr, gv[j].z, rv[j].z);
+                a.w = __fmaf_rn(lr, gv[j].w, rv[j].w);
+                st_stream(r4 + 32 * j, a);
+                flags |= (uint32_t)((__float_as_uint(a.x) & KEY_MASK) >= T0) << (4 * j);
+                flags |= (uint32_t)((__float_as_uint(a.y) & KEY_MASK) >= T0) << (4 * j + 1);
+                flags |= (uint32_t)((__float_as_uint(a.z) & KEY_MASK) >= T0) << (4 * j + 2);
+                flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0) << (4 * j + 3);
+            }
+            stream_tile_record(p, w, flags);
+        } else {
+            stream_tile_record(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi));
+        }
+        w = stat_next ? w + GW : R * GW + __shfl_sync(0xFFFFFFFFu, ticket, 0);
+    }
+}
+
+}  // namespace tke

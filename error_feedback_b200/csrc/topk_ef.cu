@@ -20,6 +20,7 @@
 #include "topk_ef.h"
 #include "common.cuh"
 #include "kernels_compress.cuh"
+#include "kernels_stream.cuh"
 #include "kernels_merge.cuh"
 #include "kernels_select.cuh"
 #include "kernels_sparse.cuh"
@@ -457,57 +458,88 @@ size_t threshold_workspace(int64_t n) {
     return compress_layout(n, plans).total;
 }
 
-// The cluster merge kernel: shared memory attribute set once per device,
-// and at least one cluster of it must fit on the device.
+// The cluster merge kernel: clusters of 16 CTAs where the device can hold
+// one (a non-portable size), else of 8; chosen once per device.
 std::mutex g_mc_mu;
-int g_mc_state[64];             // 0 unknown, 1 usable, 2 not usable
+int g_mc_cl[64];                // 0 not yet chosen, -1 neither fits, else the size
 
-int merge_cluster_ready(bool* usable) {
+template <int CL>
+cudaError_t mc_config(bool* fits) {
+    *fits = false;
+    cudaError_t e = cudaFuncSetAttribute(merge_cluster_kernel<CL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)mc_smem_bytes<CL>());
+    if (e == cudaSuccess && CL > 8)
+        e = cudaFuncSetAttribute(merge_cluster_kernel<CL>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) {
+        cudaGetLastError();            // not available on this device: try the next size
+        return cudaSuccess;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL);
+    cfg.blockDim = dim3(MC_THREADS);
+    cfg.dynamicSmemBytes = mc_smem_bytes<CL>();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, merge_cluster_kernel<CL>, &cfg);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+    }
+    *fits = clusters > 0;
+    return cudaSuccess;
+}
+
+// Cluster size for this device (0: the cluster kernel cannot run).
+int merge_cluster_size(int* cl_out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= 64) return TOPK_EF_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_mc_mu);
-    if (g_mc_state[dev] == 0) {
-        e = cudaFuncSetAttribute(merge_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(McShared));
-        if (e != cudaSuccess) return cuda_fail(e);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(MC_CL);
-        cfg.blockDim = dim3(MC_THREADS);
-        cfg.dynamicSmemBytes = sizeof(McShared);
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = MC_CL;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int clusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&clusters, merge_cluster_kernel, &cfg);
-        if (e != cudaSuccess) return cuda_fail(e);
-        g_mc_state[dev] = clusters > 0 ? 1 : 2;
+    if (g_mc_cl[dev] == 0) {
+        bool fits = false;
+        if ((e = mc_config<16>(&fits)) != cudaSuccess) return cuda_fail(e);
+        if (fits) {
+            g_mc_cl[dev] = 16;
+        } else {
+            if ((e = mc_config<8>(&fits)) != cudaSuccess) return cuda_fail(e);
+            g_mc_cl[dev] = fits ? 8 : -1;
+        }
     }
-    *usable = g_mc_state[dev] == 1;
+    *cl_out = g_mc_cl[dev] > 0 ? g_mc_cl[dev] : 0;
     return TOPK_EF_OK;
 }
 
-cudaError_t launch_merge_cluster(int32_t np, cudaStream_t st, const MergeClusterParams& cp) {
+template <int CL>
+cudaError_t launch_mc(int32_t np, cudaStream_t st, const MergeClusterParams& cp) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)np * MC_CL);
+    cfg.gridDim = dim3((unsigned)np * CL);
     cfg.blockDim = dim3(MC_THREADS);
-    cfg.dynamicSmemBytes = sizeof(McShared);
+    cfg.dynamicSmemBytes = mc_smem_bytes<CL>();
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = MC_CL;
+    attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, merge_cluster_kernel, cp);
+    return cudaLaunchKernelEx(&cfg, merge_cluster_kernel<CL>, cp);
+}
+
+cudaError_t launch_merge_cluster(int cl, int32_t np, cudaStream_t st,
+                                 const MergeClusterParams& cp) {
+    return cl == 16 ? launch_mc<16>(np, st, cp) : launch_mc<8>(np, st, cp);
 }
 
 bool bad_fp32_ptr(const void* p) { return ((uintptr_t)p & 3u) != 0; }
@@ -846,8 +878,10 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     // one cluster kernel per round when every round's merged lists fit
     bool cluster_path = !single;
     for (int r = 0; r < L.rounds; ++r)
-        cluster_path = cluster_path && L.mcap[r] <= (int64_t)MC_CL * MC_Q;
-    if (cluster_path && (rc = merge_cluster_ready(&cluster_path)) != TOPK_EF_OK) return rc;
+        cluster_path = cluster_path && L.mcap[r] <= MC_PAIR_MAX;
+    int mc_cl = 0;
+    if (cluster_path && (rc = merge_cluster_size(&mc_cl)) != TOPK_EF_OK) return rc;
+    cluster_path = cluster_path && mc_cl > 0;
     const uint32_t kernels =
         single ? 2u : (uint32_t)(cluster_path ? 1 + L.rounds : 1 + 2 * L.rounds);
 
@@ -942,7 +976,7 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
             cp.n_bad = r == 0 ? (int32_t)L.vblocks : 0;
             cp.ctrl = ctrl;
             trace_before(st, "merge_cluster_kernel");
-            e = launch_merge_cluster(L.np[r], st, cp);
+            e = launch_merge_cluster(mc_cl, L.np[r], st, cp);
             trace_after(st);
             if (e != cudaSuccess) return cuda_fail(e);
         }
