@@ -72,6 +72,9 @@ struct McFixed {
     int64_t part[2];
     uint32_t live, above, nlist, gt, eq, pg, pe;
     uint32_t loff[17];                                // list offsets by cluster rank
+    uint32_t lcnt[16];                                // list lengths by cluster rank
+    __align__(16) uint32_t hslice[D1_BINS / 8];       // this CTA's slice of the summed h1
+    uint32_t live_tot;
     uint32_t E, pre_above;
     FindResult fr;
 };
@@ -169,6 +172,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     for (int i = tid; i < D1_BINS; i += blockDim.x) S.h1[i] = 0;
     for (int i = tid; i < D2_BINS; i += blockDim.x) S.h2[i] = 0;
     for (int i = tid; i < D3_BINS; i += blockDim.x) S.h3[i] = 0;
+    for (int i = tid; i < D1_BINS / CL; i += blockDim.x) S.hslice[i] = 0;
     __syncthreads();
     if (stamp) p.ctrl->t_phase[1] = global_ns();
     const int64_t i0 = S.part[0], i1 = max(S.part[1], i0);
@@ -269,14 +273,38 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     cl.sync();                                           // [1] h1 and live of every CTA
     if (stamp) p.ctrl->t_phase[4] = global_ns();
 
-    uint32_t live_tot = 0;
-#pragma unroll
-    for (int r = 0; r < CL; ++r) live_tot += *cl.map_shared_rank(&S.live, r);
+    // live entries of the pair (warp 0, lane r reads rank r), and this CTA's
+    // slice of the summed digit-1 histogram: bins [cr*SB, cr*SB + SB) over
+    // all CTAs, one 16-byte remote load per thread
+    constexpr int SB = D1_BINS / CL;
+    if (tid < 32) {
+        const uint32_t lv = tid < CL ? *cl.map_shared_rank(&S.live, tid) : 0u;
+        const uint32_t lt = warp_sum(lv);
+        if (tid == 0) S.live_tot = lt;
+    }
+    for (int t = tid; t < (SB / 4) * CL; t += blockDim.x) {
+        const int r = t / (SB / 4), j = t - r * (SB / 4);
+        const uint4 v = *reinterpret_cast<const uint4*>(cl.map_shared_rank(S.h1 + cr * SB + 4 * j, r));
+        atomicAdd(&S.hslice[4 * j + 0], v.x);
+        atomicAdd(&S.hslice[4 * j + 1], v.y);
+        atomicAdd(&S.hslice[4 * j + 2], v.z);
+        atomicAdd(&S.hslice[4 * j + 3], v.w);
+    }
+    cl.sync();                                           // [1b] every slice summed
+    const uint32_t live_tot = S.live_tot;
     const uint32_t kp = live_tot < p.kmax ? live_tot : p.kmax;
     uint32_t b1 = 0, rem = kp;
     bool ok = kp > 0;
     if (kp > 0) {
-        cluster_find<CL, D1_BINS>(cl, S, S.h1, rem);
+        // the summed histogram from its CL owners, 16 bytes per thread
+        for (int t = tid; t < D1_BINS / 4; t += blockDim.x) {
+            const int r = (4 * t) / SB;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                cl.map_shared_rank(S.hslice + (4 * t - r * SB), r));
+            reinterpret_cast<uint4*>(S.tot)[t] = v;
+        }
+        __syncthreads();
+        block_find_bin(S.tot, D1_BINS, rem, S.red, &S.fr);
         ok = S.fr.ok;
         b1 = S.fr.bin;
         rem -= S.fr.above;
@@ -312,7 +340,9 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     cl.sync();                                           // [2] every CTA's list and count
     if (stamp) p.ctrl->t_phase[5] = global_ns();
 
-    // list lengths and counts above b1 of all CTAs (lane r reads rank r)
+    // list lengths and counts above b1 of all CTAs (lane r reads rank r);
+    // in the gathered list each CTA's entries start at a multiple of 4
+    constexpr uint32_t SENT = 0xFFFFFFFFu;              // padding entry
     if (tid < 32) {
         const uint32_t lane = lane_id();
         uint32_t nr = 0, ar = 0;
@@ -320,8 +350,12 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             nr = *cl.map_shared_rank(&S.nlist, (int)lane);
             ar = *cl.map_shared_rank(&S.above, (int)lane);
         }
-        const uint32_t incl = warp_incl_scan(nr);
-        if (lane < (uint32_t)CL) S.loff[lane] = incl - nr;
+        const uint32_t np4 = (nr + 3u) & ~3u;
+        const uint32_t incl = warp_incl_scan(np4);
+        if (lane < (uint32_t)CL) {
+            S.loff[lane] = incl - np4;
+            S.lcnt[lane] = nr;
+        }
         if (lane == (uint32_t)CL - 1) S.loff[CL] = incl;
         const uint32_t pa = warp_sum((int)lane < cr ? ar : 0u);
         const uint32_t all = __shfl_sync(0xFFFFFFFFu, incl, 31);
@@ -335,36 +369,31 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     uint32_t T = NO_KEY, q = 0, pg = 0, pe = 0;
     const bool gathered = E <= (uint32_t)C::GCAP;       // the same in every CTA
     if (gathered) {
-        // all lists, in cluster rank order: batches of GU independent
-        // remote loads per thread
-        constexpr int GU = 8;
-        for (uint32_t g0 = tid; g0 < E; g0 += GU * blockDim.x) {
-            uint32_t v[GU];
+        // all lists, in cluster rank order, 16 bytes per remote load
+        uint4* g4 = reinterpret_cast<uint4*>(glist);
+        for (uint32_t u = tid; u < E / 4; u += blockDim.x) {
+            int r = 0;
 #pragma unroll
-            for (int u = 0; u < GU; ++u) {
-                const uint32_t g = g0 + u * blockDim.x;
-                v[u] = 0;
-                if (g < E) {
-                    int r = 0;
-#pragma unroll
-                    for (int st = CL / 2; st >= 1; st >>= 1)
-                        if (r + st < CL && S.loff[r + st] <= g) r += st;
-                    v[u] = *cl.map_shared_rank(mylist + (g - S.loff[r]), r);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < GU; ++u)
-                if (g0 + u * blockDim.x < E) glist[g0 + u * blockDim.x] = v[u];
+            for (int st = CL / 2; st >= 1; st >>= 1)
+                if (r + st < CL && S.loff[r + st] <= 4 * u) r += st;
+            const uint32_t i = 4 * u - S.loff[r];          // first entry of the load
+            uint4 v = *reinterpret_cast<const uint4*>(cl.map_shared_rank(mylist + i, r));
+            const uint32_t nr = S.lcnt[r];
+            if (i + 0 >= nr) v.x = SENT;
+            if (i + 1 >= nr) v.y = SENT;
+            if (i + 2 >= nr) v.z = SENT;
+            if (i + 3 >= nr) v.w = SENT;
+            g4[u] = v;
         }
         if (kp > 0 && ok) {
             // bits 19..10, then 9..0 of the k-th key inside bin b1
-            list_find(S, glist, E, 1024, rem, [](uint32_t) { return true; },
+            list_find(S, glist, E, 1024, rem, [](uint32_t v) { return v != 0xFFFFFFFFu; },
                       [](uint32_t v) { return (v >> 10) & 1023u; });
             const uint32_t bA = S.fr.bin;
             const uint32_t remA = rem - S.fr.above;
             ok = S.fr.ok;
             list_find(S, glist, E, 1024, remA,
-                      [bA](uint32_t v) { return ((v >> 10) & 1023u) == bA; },
+                      [bA](uint32_t v) { return v != 0xFFFFFFFFu && ((v >> 10) & 1023u) == bA; },
                       [](uint32_t v) { return v & 1023u; });
             ok = ok && S.fr.ok;
             const uint32_t t = (bA << 10) | S.fr.bin;
