@@ -80,6 +80,7 @@ struct SelShared {
     uint32_t pre[4];
     uint64_t ovf_pos[SEL_THREADS];   // gather: output position of each overflow tile
     uint64_t before;                 // gather: output offset of the block
+    uint64_t total;                  // gather (look-all): candidates of all blocks
 };
 
 // Block-wide copy of n words (n a multiple of 4, 16-byte aligned) into
@@ -177,6 +178,7 @@ struct CompressSrc {
     uint32_t* ent;               // [T][ENT_PER] entry lists
     uint32_t* ent_cnt;           // [T] their lengths
     uint64_t* agg;               // [grid] each block's candidate count + 1 (0: not yet)
+    int32_t r1_done;             // one tensor: the streaming pass built relative digit 1
     int32_t force_dense;
     int32_t dense;               // decided inside the kernel
 
@@ -462,7 +464,7 @@ __device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelSh
             src.cand_val[q] = t.v[i];
             if (kThr) src.resid[e] = 0.0f;
         }
-        if (!kThr) r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), t.v[i], s_r1);
+        if (!kThr && !src.r1_done) r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), t.v[i], s_r1);
     }
 }
 
@@ -491,6 +493,37 @@ __device__ uint64_t look_back(const uint64_t* agg, int c, uint32_t* status, SelS
     }
     __syncthreads();
     return S.before;
+}
+
+// Output offset of block c and the total of all blocks (warp 0 reads every
+// published count; all blocks publish before any heavy work, so the wait is
+// short; bounded all the same).  Results in S.before and S.total.
+__device__ void look_all(const uint64_t* agg, int c, uint32_t* status, SelShared& S) {
+    if (threadIdx.x < 32) {
+        uint64_t before = 0, total = 0;
+        for (int j = (int)lane_id(); j < (int)gridDim.x; j += 32) {
+            uint64_t v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
+            uint32_t it = 0;
+            while (v == 0) {
+                if (++it > SPIN_LIMIT) {
+                    atomicOr(status, ST_TIMEOUT);
+                    break;
+                }
+                __nanosleep(32);
+                v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
+            }
+            const uint64_t cnt = v ? v - 1 : 0;
+            total += cnt;
+            if (j < c) before += cnt;
+        }
+        before = warp_sum(before);
+        total = warp_sum(total);
+        if (threadIdx.x == 0) {
+            S.before = before;
+            S.total = total;
+        }
+    }
+    __syncthreads();
 }
 
 // Gather a warp tile with more than WT_CAP candidates (one warp): rescan it
@@ -531,7 +564,7 @@ __device__ void gather_rescan(const CompressSrc& src, const SelShared& S, uint32
                 src.cand_val[q] = v[u];
                 if (kThr) src.resid[e] = 0.0f;
             }
-            if (!kThr) r1_add(src, S, l, v[u], s_r1);
+            if (!kThr && !src.r1_done) r1_add(src, S, l, v[u], s_r1);
         }
         pos += __popc(m);
     }
@@ -589,7 +622,7 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
     // relative digit 1 in shared memory when the whole chunk is in one tensor
     const int64_t e0 = (int64_t)w0 * WT, e1 = min((int64_t)w1 * WT, src.N);
     const int lc = w0 < w1 ? seg_of(s_off, T, e0) : 0;
-    const bool one = !kThr && w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
+    const bool one = !kThr && !src.r1_done && w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
     uint32_t* s_r1 = one ? S.stage : nullptr;
     if (one)
         for (int i = tid; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
@@ -607,7 +640,12 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
         const bool staged = cnt > 0 && cnt <= (uint32_t)WT_CAP;
         if (staged) load_staged(src, w, cnt, tc);
         if (!have_before) {
-            before = look_back(src.agg, c, status, S);
+            if (src.r1_done) {
+                look_all(src.agg, c, status, S);
+                before = S.before;
+            } else {
+                before = look_back(src.agg, c, status, S);
+            }
             have_before = true;
             mark_phase(cm.ctrl, 4);
         }
@@ -657,18 +695,27 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
 __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t& epoch,
                                 SelShared& S, uint64_t& my0, uint64_t& my1) {
     gather_phase<false>(src, cm, S, my0, my1);
-    if (!grid_barrier(cm.bar, epoch, &cm.ctrl->status, &S.flag)) return false;
-    mark_phase(cm.ctrl, 1);
-
     const int T = src.T;
     const int tid = threadIdx.x;
-    const uint64_t total = (uint64_t)src.cand_start[T];
-    const bool fits = total <= src.cap;
+    uint64_t total;
     uint32_t bad = 0;
-    for (int l = tid; l < T; l += blockDim.x)
-        bad |= ((uint64_t)(src.cand_start[l + 1] - src.cand_start[l]) < (uint64_t)src.meta[l].k) ||
-               src.rel_overflow(l);
-    bad = block_sum(bad, S.red);
+    if (src.r1_done) {
+        // one tensor, relative digit 1 built by the streaming pass and the
+        // total known from the look-all: no barrier needed to decide
+        total = S.total;
+        bad = (total < (uint64_t)src.meta[0].k) || src.rel_overflow(0);
+        mark_phase(cm.ctrl, 1);
+    } else {
+        if (!grid_barrier(cm.bar, epoch, &cm.ctrl->status, &S.flag)) return false;
+        mark_phase(cm.ctrl, 1);
+        total = (uint64_t)src.cand_start[T];
+        for (int l = tid; l < T; l += blockDim.x)
+            bad |= ((uint64_t)(src.cand_start[l + 1] - src.cand_start[l]) <
+                    (uint64_t)src.meta[l].k) ||
+                   src.rel_overflow(l);
+        bad = block_sum(bad, S.red);
+    }
+    const bool fits = total <= src.cap;
     src.dense = (src.force_dense || !fits || bad) ? 1 : 0;
     if (blockIdx.x == 0 && tid == 0) {
         cm.ctrl->mode = src.dense;
@@ -756,7 +803,16 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
     const int T = src.T;
     uint32_t* status = &cm.ctrl->status;
     __syncthreads();
-    for (int l = tid; l <= T; l += blockDim.x) S.seg[l] = src.cand_start[l];
+    if (src.r1_done) {
+        // one tensor: [0, total), the total from the look-all (cand_start[1]
+        // is written by the last block and not yet ordered by a barrier)
+        if (tid == 0) {
+            S.seg[0] = 0;
+            S.seg[1] = (int64_t)S.total;
+        }
+    } else {
+        for (int l = tid; l <= T; l += blockDim.x) S.seg[l] = src.cand_start[l];
+    }
     __syncthreads();
     const bool has = a1 > a0;
     // an empty range passes the tensor running through it on to the next block

@@ -22,6 +22,7 @@ struct StreamParams {
     Ctrl* ctrl;
     uint32_t* wt_count;     // [num_wt] candidates of each warp tile (exact)
     uint16_t* wt_off;       // [num_wt][WT_CAP]: their offsets in the tile, unordered
+    uint32_t* r1;           // one tensor: its candidates' relative digit-1 histogram
 };
 
 // Tensor l with off[l] <= e < off[l+1] (empty tensors are skipped).
@@ -47,14 +48,21 @@ __device__ __forceinline__ int lower_bound_off(const int64_t* off, int T, int64_
 struct StreamShared {
     int64_t off[TCAP_LARGE + 1];
     uint32_t T0[TCAP_LARGE];
+    uint32_t r1[REL_BINS];      // one tensor: this block's share of p.r1
 };
+
+// Relative digit-1 bin of a candidate (key >= T0): min((key - T0) >> sh, 4095).
+__device__ __forceinline__ uint32_t stream_rel_bin(float a, uint32_t T0, uint32_t sh) {
+    return min((key_of(a) - T0) >> sh, (uint32_t)(REL_BINS - 1));
+}
 
 // General warp tile: a partial last tile, a tile that spans tensors, or
 // unaligned inputs.  Computes acc, stores it, returns the candidate flags
 // (bit 4j + v for element base + 128 j + 4 lane + v).
 template <bool VEC>
-__device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, const StreamShared& S,
-                                                     int64_t base, int l_lo, int l_hi) {
+__device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, StreamShared& S,
+                                                     int64_t base, int l_lo, int l_hi,
+                                                     uint32_t sh) {
     const uint32_t lane = lane_id();
     uint32_t flags = 0;
     for (int j = 0; j < WT_VECS; ++j) {
@@ -81,7 +89,10 @@ __device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, cons
             if (e + v >= p.N) continue;
             int l = l_lo;
             while (l < l_hi && S.off[l + 1] <= e + v) ++l;
-            if (key_of(a[v]) >= S.T0[l]) flags |= 1u << (j * 4 + v);
+            if (key_of(a[v]) >= S.T0[l]) {
+                flags |= 1u << (j * 4 + v);
+                if (p.r1) atomicAdd(&S.r1[stream_rel_bin(a[v], S.T0[l], sh)], 1u);
+            }
         }
     }
     return flags;
@@ -154,6 +165,11 @@ stream_kernel(const __grid_constant__ StreamParams p) {
         S.T0[l] = p.meta[l].T0;
     }
     if (tid == 0) S.off[T] = p.N;
+    // one tensor: the candidates' relative digit-1 histogram is built here
+    const bool hist = flat && p.r1 != nullptr;
+    const uint32_t sh = hist ? p.meta[0].shift : 0u;
+    if (hist)
+        for (int i = tid; i < REL_BINS; i += blockDim.x) S.r1[i] = 0;
     __syncthreads();
 
     // Warp tiles are handed out statically for all but the last rounds, then
@@ -204,12 +220,29 @@ stream_kernel(const __grid_constant__ StreamParams p) {
                 flags |= (uint32_t)((__float_as_uint(a.y) & KEY_MASK) >= T0) << (4 * j + 1);
                 flags |= (uint32_t)((__float_as_uint(a.z) & KEY_MASK) >= T0) << (4 * j + 2);
                 flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0) << (4 * j + 3);
+                rv[j] = a;
             }
             stream_tile_record(p, w, flags);
+            if (hist && flags) {
+#pragma unroll
+                for (int j = 0; j < WT_VECS; ++j) {
+                    if ((flags >> (4 * j)) & 0xFu) {
+                        if ((flags >> (4 * j)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].x, T0, sh)], 1u);
+                        if ((flags >> (4 * j + 1)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].y, T0, sh)], 1u);
+                        if ((flags >> (4 * j + 2)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].z, T0, sh)], 1u);
+                        if ((flags >> (4 * j + 3)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].w, T0, sh)], 1u);
+                    }
+                }
+            }
         } else {
-            stream_tile_record(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi));
+            stream_tile_record(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi, sh));
         }
         w = stat_next ? w + GW : R * GW + __shfl_sync(0xFFFFFFFFu, ticket, 0);
+    }
+    if (hist) {
+        __syncthreads();
+        for (int i = tid; i < REL_BINS; i += blockDim.x)
+            if (S.r1[i]) atomicAdd(&p.r1[i], S.r1[i]);
     }
 }
 

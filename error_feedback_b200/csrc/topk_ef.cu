@@ -319,7 +319,8 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
 // The streaming pass of one group (after its setup kernel, with
 // programmatic serialisation); fills *sp for the select kernels.
 cudaError_t launch_stream(const Group& g, const CLayout& L, char* ws, const float* gg, float* rg,
-                          float lr, cudaStream_t st, const DevFacts& f, StreamParams* sp_out) {
+                          float lr, cudaStream_t st, const DevFacts& f, StreamParams* sp_out,
+                          bool build_r1) {
     StreamParams sp;
     sp.grad = gg;
     sp.resid = rg;
@@ -331,6 +332,10 @@ cudaError_t launch_stream(const Group& g, const CLayout& L, char* ws, const floa
     sp.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
     sp.wt_count = reinterpret_cast<uint32_t*>(ws + L.wt_count);
     sp.wt_off = reinterpret_cast<uint16_t*>(ws + L.wt_off);
+    // one tensor: the streaming pass builds the candidates' relative digit 1
+    sp.r1 = build_r1 && g.plans.size() == 1
+                ? reinterpret_cast<uint32_t*>(ws + L.hist) + CH_R1
+                : nullptr;
     *sp_out = sp;
     const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
     const int64_t warps_needed = L.num_wt;
@@ -384,13 +389,19 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     if (e != cudaSuccess) return cuda_fail(e);
     if (g.N == 0) return TOPK_EF_OK;
 
+    // a single tensor with a short candidate list: the streaming pass builds
+    // relative digit 1 and the select kernel saves a grid barrier; long
+    // lists would pay more in the streaming pass than the barrier costs
+    const bool build_r1 = T == 1 && L.cap <= ((int64_t)1 << 19);
     StreamParams sp;
-    if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp)) != cudaSuccess) return cuda_fail(e);
+    if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp, build_r1)) != cudaSuccess)
+        return cuda_fail(e);
     Ctrl* ctrl = sp.ctrl;
 
     CompressSrc src = make_src(g, L, ws, sp, rg);
     src.out_idx = out_idx;
     src.out_val = out_val;
+    src.r1_done = sp.r1 != nullptr ? 1 : 0;
     src.force_dense = force_dense ? 1 : 0;
     src.dense = 0;
     SelCommon cm;
@@ -433,7 +444,7 @@ int threshold_call(const float* grad, float* resid, int64_t n, float lr, uint32_
         return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
     }
     StreamParams sp;
-    if ((e = launch_stream(g, L, ws, grad, resid, lr, st, f, &sp)) != cudaSuccess)
+    if ((e = launch_stream(g, L, ws, grad, resid, lr, st, f, &sp, false)) != cudaSuccess)
         return cuda_fail(e);
     CompressSrc src = make_src(g, L, ws, sp, resid);
     src.cand_idx = reinterpret_cast<uint32_t*>(out_idx);
