@@ -137,9 +137,9 @@ ag_bounds_kernel(const __grid_constant__ AllGatherParams p) {
     if (__any_sync(0xFFFFFFFFu, bad) && lane_id() == 0) atomicOr(&p.ctrl->status, ST_BAD_INPUT);
 }
 
-// Bound b of row r: the table's entry, or (left unset) a binary search.
-__device__ __forceinline__ uint32_t ag_bound(const AllGatherParams& p, int64_t r, int64_t b) {
-    const uint32_t v = p.bound[r * (p.nchunks + 1) + b];
+// Bound b of row r from the table's entry v, or (left unset) a binary search.
+__device__ __forceinline__ uint32_t ag_bound(const AllGatherParams& p, int64_t r, int64_t b,
+                                             uint32_t v) {
     if (v != AG_UNSET) return v < (uint32_t)p.k_in ? v : (uint32_t)p.k_in;
     const int32_t* row = p.idx + r * p.k_in;
     const int64_t key = b * AG_CHUNK;
@@ -180,24 +180,43 @@ ag_sum_kernel(const __grid_constant__ AllGatherParams p) {
     uint32_t* base = lo + P;                    // [P + 1]
     const int64_t nw = (int64_t)gridDim.x * AG_WARPS;
     // each lane scans the rows [per * lane, per * lane + per)
+    constexpr int PER_MAX = AG_MAX_P / 32;
     const int per = (P + 31) / 32;
-    for (int64_t c = (int64_t)blockIdx.x * AG_WARPS + warp_id(); c < p.nchunks; c += nw) {
+    const int64_t nb = p.nchunks + 1;
+    // raw table bounds of this warp's next chunk, loaded one chunk ahead
+    uint32_t ta[PER_MAX], tb[PER_MAX];
+    auto fetch = [&](int64_t c) {
+#pragma unroll
+        for (int k = 0; k < PER_MAX; ++k) {
+            const int r = per * (int)lane + k;
+            ta[k] = tb[k] = AG_UNSET;
+            if (k < per && r < P && c < p.nchunks) {
+                ta[k] = p.bound[r * nb + c];
+                tb[k] = p.bound[r * nb + c + 1];
+            }
+        }
+    };
+    int64_t c = (int64_t)blockIdx.x * AG_WARPS + warp_id();
+    fetch(c);
+    for (; c < p.nchunks; c += nw) {
         const int64_t c0 = c * AG_CHUNK;
         const int len = (int)(p.n - c0 < AG_CHUNK ? p.n - c0 : AG_CHUNK);
 #pragma unroll
         for (int i = 0; i < AG_CHUNK / 128; ++i)
             reinterpret_cast<float4*>(acc)[lane + 32 * i] = make_float4(0.f, 0.f, 0.f, 0.f);
         uint32_t run = 0;
-        for (int k = 0; k < per; ++k) {
+#pragma unroll
+        for (int k = 0; k < PER_MAX; ++k) {
             const int r = per * (int)lane + k;
-            if (r >= P) break;
-            const uint32_t a = ag_bound(p, r, c);
-            uint32_t b = ag_bound(p, r, c + 1);
+            if (k >= per || r >= P) continue;
+            const uint32_t a = ag_bound(p, r, c, ta[k]);
+            uint32_t b = ag_bound(p, r, c + 1, tb[k]);
             if (b < a) b = a;
             lo[r] = a;
             base[r] = run;                          // local prefix, fixed below
             run += b - a;
         }
+        fetch(c + nw);
         const uint32_t incl = warp_incl_scan(run);
         const uint32_t add = incl - run;
         for (int k = 0; k < per; ++k) {
