@@ -52,6 +52,7 @@ TRACE_EVERY = 8            # timed region: events around every 8th dominant laun
 LR = np.float32(0.1)
 POOL = 4          # distinct gradients cycled through the steps
 KERNEL_SOURCES = ["error_feedback_b200/csrc/kernels_stream.cuh",
+                  "error_feedback_b200/csrc/kernels_compress.cuh",
                   "error_feedback_b200/csrc/common.cuh"]
 
 

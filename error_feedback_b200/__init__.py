@@ -360,10 +360,10 @@ def topk_ef_last_device_status(ws, stream=None) -> int:
 
 
 def topk_ef_path_info(ws, stream=None) -> dict:
-    info = (ctypes.c_int64 * 4)()
+    info = (ctypes.c_int64 * 6)()
     _check(lib().topk_ef_path_info(ws.data_ptr(), _stream(stream), info), "topk_ef_path_info")
     return {"fallback": int(info[0]), "candidates": int(info[1]), "capacity": int(info[2]),
-            "kernels": int(info[3])}
+            "kernels": int(info[3]), "crowded_bin": int(info[4])}
 
 
 def topk_ef_phase_times(ws, stream=None) -> list:

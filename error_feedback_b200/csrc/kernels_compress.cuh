@@ -29,7 +29,8 @@ constexpr int SAMPLE_BINS = 4096;    // key >> 19
 constexpr int K1_THREADS = 256;
 constexpr int WT = 1024;             // elements per warp tile
 constexpr int WT_VECS = WT / 128;    // float4 of each input per lane per warp tile
-constexpr int WT_CAP = 16;           // candidate offsets staged per warp tile
+constexpr int WT_CAP = 32;           // candidate offsets staged per warp tile
+constexpr int WT_THREAD = 16;        // staged candidates the select gathers per thread
 constexpr uint32_t STREAM_PREFETCH = 3;   // warp tiles per warp pulled into L2 early
 constexpr int ZERO_THREADS = 1024;
 

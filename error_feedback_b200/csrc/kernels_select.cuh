@@ -417,8 +417,8 @@ __device__ __forceinline__ void r1_add(const CompressSrc& src, const SelShared& 
 // slots >= cnt hold 0xFFFF, above every offset) and the values read back
 // from the residual (which holds acc).
 struct TileCands {
-    uint32_t o[WT_CAP];
-    float v[WT_CAP];
+    uint32_t o[WT_THREAD];
+    float v[WT_THREAD];
 };
 
 __device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, uint32_t cnt,
@@ -433,7 +433,7 @@ __device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, 
     t.o[12] = b.z & 0xFFFFu; t.o[13] = b.z >> 16; t.o[14] = b.w & 0xFFFFu; t.o[15] = b.w >> 16;
     const int64_t base = (int64_t)w * WT;
 #pragma unroll
-    for (int i = 0; i < WT_CAP; ++i) {
+    for (int i = 0; i < WT_THREAD; ++i) {
         if ((uint32_t)i >= cnt) t.o[i] = 0xFFFFu;
         t.v[i] = (uint32_t)i < cnt ? src.resid[base + t.o[i]] : 0.f;
     }
@@ -526,6 +526,31 @@ __device__ void look_all(const uint64_t* agg, int c, uint32_t* status, SelShared
     __syncthreads();
 }
 
+// Gather a warp tile with WT_THREAD < cnt <= WT_CAP staged candidates (one
+// warp): lane i takes offset i, ranks it among the others by shuffles and
+// reads its value back from the residual.
+template <bool kThr>
+__device__ void gather_warp_staged(const CompressSrc& src, const SelShared& S, uint32_t w,
+                                   uint64_t pos, uint32_t cnt, uint32_t* s_r1, int lc) {
+    const uint32_t lane = lane_id();
+    const int64_t base = (int64_t)w * WT;
+    const uint32_t o = lane < cnt ? (uint32_t)src.wt_off[(size_t)w * WT_CAP + lane] : 0xFFFFu;
+    uint32_t rank = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rank += __shfl_sync(0xFFFFFFFFu, o, i) < o;
+    if (lane < cnt) {
+        const int64_t e = base + o;
+        const float v = src.resid[e];
+        const uint64_t q = pos + rank;
+        if (q < src.cap) {
+            src.cand_idx[q] = (uint32_t)e;
+            src.cand_val[q] = v;
+            if (kThr) src.resid[e] = 0.0f;
+        }
+        if (!kThr && !src.r1_done) r1_add(src, S, s_r1 ? lc : seg_of(S.seg, src.T, e), v, s_r1);
+    }
+}
+
 // Gather a warp tile with more than WT_CAP candidates (one warp): rescan it
 // from the residual (which holds acc) with the streaming pass's test.  The
 // 32 coalesced loads of the tile (element base + 32 u + lane) are issued at
@@ -589,8 +614,9 @@ __device__ uint32_t tile_count_below(const CompressSrc& src, const SelShared& S,
 // of warp tiles, publishes its candidate count at once and finds its output
 // offset by looking back at the counts of the blocks before it (no grid
 // barrier).  It copies its candidates, in index order, to [my0, my1) of the
-// dense list (the staged ones from registers loaded before the look-back;
-// tiles with more than WT_CAP candidates are rescanned), builds the relative
+// dense list (up to WT_THREAD staged ones per tile from registers loaded
+// before the look-back; up to WT_CAP by a warp; more by a rescan of the
+// tile), builds the relative
 // digit-1 histograms (not in threshold mode) and records where each
 // tensor's candidates start.
 template <bool kThr>
@@ -626,7 +652,7 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
     uint32_t* s_r1 = one ? S.stage : nullptr;
     if (one)
         for (int i = tid; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
-    // tiles with more than WT_CAP candidates of a piece: (tile, position)
+    // tiles with more than WT_THREAD candidates of a piece: (tile, position)
     uint32_t* s_ovf_w = S.h1;
     uint64_t before = 0, run = 0;
     bool have_before = false;
@@ -637,7 +663,7 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
         uint32_t piece;
         const uint32_t ex = block_excl_scan(cnt, S.red, &piece);
         TileCands tc;
-        const bool staged = cnt > 0 && cnt <= (uint32_t)WT_CAP;
+        const bool staged = cnt > 0 && cnt <= (uint32_t)WT_THREAD;
         if (staged) load_staged(src, w, cnt, tc);
         if (!have_before) {
             if (src.r1_done) {
@@ -656,19 +682,24 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
             for (int l = max(1, lower_bound_off(s_off, T, base)); l < T && s_off[l] < tend; ++l)
                 src.cand_start[l] = (int64_t)(pos + tile_count_below(src, S, w, cnt, s_off[l]));
         }
-        if (cnt > (uint32_t)WT_CAP) {
+        if (cnt > (uint32_t)WT_THREAD) {
             const uint32_t slot = atomicAdd(reinterpret_cast<uint32_t*>(&S.flag), 1u);
             s_ovf_w[slot] = w;
             S.ovf_pos[slot] = pos;
         } else if (cnt > 4) {
-            store_ranked<WT_CAP, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
+            store_ranked<WT_THREAD, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         } else if (cnt > 0) {
             store_ranked<4, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         }
         __syncthreads();
         const uint32_t novf = (uint32_t)S.flag;
-        for (uint32_t i = warp; i < novf; i += nwarps)
-            gather_rescan<kThr>(src, S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
+        for (uint32_t i = warp; i < novf; i += nwarps) {
+            const uint32_t wo = s_ovf_w[i];
+            if (src.wt_count[wo] <= (uint32_t)WT_CAP)
+                gather_warp_staged<kThr>(src, S, wo, S.ovf_pos[i], src.wt_count[wo], s_r1, lc);
+            else
+                gather_rescan<kThr>(src, S, wo, S.ovf_pos[i], s_r1, lc);
+        }
         __syncthreads();
         run += piece;
     }
@@ -788,6 +819,72 @@ __device__ __forceinline__ void zero_stage(SelShared& S) {
     __syncthreads();
 }
 
+// A tensor whose candidates [a, b) all lie in this block's range, at most
+// EMIT_TILE of them: selected from registers alone (the candidates are read
+// once; both relative digits are histogrammed locally) and emitted.  Returns
+// false if the counts do not add up.
+__device__ bool local_small(const CompressSrc& src, int l, int64_t a, int64_t b, SelShared& S) {
+    const int tid = threadIdx.x;
+    const uint32_t k = src.meta[l].k;
+    const uint32_t T0 = S.T0[l], sh = S.shift[l];
+    const uint32_t lmask = (1u << sh) - 1u;
+    uint32_t idx[EMIT_PER_THREAD], key[EMIT_PER_THREAD], bin[EMIT_PER_THREAD];
+    float val[EMIT_PER_THREAD];
+#pragma unroll
+    for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+        const int64_t pos = a + (int64_t)tid * EMIT_PER_THREAD + u;
+        idx[u] = DEAD;
+        val[u] = 0.f;
+        if (pos < b) {
+            idx[u] = src.cand_idx[pos];
+            val[u] = src.cand_val[pos];
+        }
+        key[u] = key_of(val[u]);
+        bin[u] = min((key[u] - T0) >> sh, (uint32_t)(REL_BINS - 1));
+    }
+    if (k == 0) return true;
+    zero_stage(S);
+#pragma unroll
+    for (int u = 0; u < EMIT_PER_THREAD; ++u)
+        if (idx[u] != DEAD) atomicAdd(&S.stage[bin[u]], 1u);
+    __syncthreads();
+    block_find_bin(S.stage, REL_BINS, k, S.red, &S.fr);
+    if (!S.fr.ok) return false;
+    const uint32_t b1 = S.fr.bin, rem = k - S.fr.above;
+    zero_stage(S);
+#pragma unroll
+    for (int u = 0; u < EMIT_PER_THREAD; ++u)
+        if (idx[u] != DEAD && bin[u] == b1) atomicAdd(&S.stage[(key[u] - T0) & lmask], 1u);
+    __syncthreads();
+    block_find_bin(S.stage, REL_BINS, rem, S.red, &S.fr);
+    if (!S.fr.ok) return false;
+    const uint32_t Tk = T0 + (b1 << sh) + S.fr.bin;
+    const uint32_t q = rem - S.fr.above;
+    uint32_t cls = 0;   // bit u: gt, bit 4+u: eq
+#pragma unroll
+    for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+        if (idx[u] == DEAD) continue;
+        if (key[u] > Tk) cls |= 1u << u;
+        else if (key[u] == Tk) cls |= 1u << (4 + u);
+    }
+    const uint64_t mine = ((uint64_t)__popc(cls & 0xFu) << 32) | (uint64_t)__popc(cls >> 4);
+    uint64_t tot;
+    const uint64_t ex = block_excl_scan(mine, S.scan, &tot);
+    uint32_t g = (uint32_t)(ex >> 32), e = (uint32_t)(ex & 0xFFFFFFFFu);
+#pragma unroll
+    for (int u = 0; u < EMIT_PER_THREAD; ++u) {
+        if ((cls >> u) & 1u) {
+            const uint32_t rank = g + (e < q ? e : q);
+            if (rank < k) src.emit(l, rank, idx[u], val[u]);
+            ++g;
+        } else if ((cls >> (4 + u)) & 1u) {
+            if (e < q) src.emit(l, g + e, idx[u], val[u]);
+            ++e;
+        }
+    }
+    return true;
+}
+
 // Selection and emission on the dense candidate list.  The block's range
 // [a0, a1) is what it gathered.  A tensor that lies wholly inside the range
 // is finished here alone.  For the (at most two) tensors that cross the
@@ -825,12 +922,16 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
         const int64_t b = min((int64_t)a1, S.seg[l + 1]);
         if (a >= b) continue;
         const uint32_t k = src.meta[l].k;
+        const bool local = S.seg[l] >= (int64_t)a0 && S.seg[l + 1] <= (int64_t)a1;
+        if (local && b - a <= (int64_t)EMIT_TILE) {
+            if (!local_small(src, l, a, b, S) && tid == 0) atomicOr(status, ST_INCONSISTENT);
+            continue;
+        }
         const RelState rs = resolve_rel1(src.h(l, CH_R1), k, S);
         if (!rs.ok) {
             if (k && tid == 0) atomicOr(status, ST_INCONSISTENT);
             continue;
         }
-        const bool local = S.seg[l] >= (int64_t)a0 && S.seg[l + 1] <= (int64_t)a1;
         if (local) {
             zero_stage(S);
             scan_rel_bin(src, l, a, b, rs, false, S);

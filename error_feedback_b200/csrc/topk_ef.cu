@@ -1065,6 +1065,8 @@ int topk_ef_path_info(const void* ws, void* stream, int64_t* info) {
     info[1] = (int64_t)c.cand_total;
     info[2] = (int64_t)c.cap;
     info[3] = c.kernels;
+    info[4] = c.r2_path ? 1 : 0;
+    info[5] = 0;
     return TOPK_EF_OK;
 }
 

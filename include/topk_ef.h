@@ -285,7 +285,11 @@ const char* topk_ef_status_string(int status);
  *   info[1]  candidates kept by the prefilter
  *   info[2]  candidate capacity of the workspace
  *   info[3]  kernels launched by that call
- * `info` is host memory of 4 int64.  Returns a status code.
+ *   info[4]  1 if the k-th key's relative digit-1 bin of some tensor held
+ *            more candidates than its entry list, so the select kernel took
+ *            the exact-count exchange (one more grid barrier); else 0
+ *   info[5]  reserved (0)
+ * `info` is host memory of 6 int64.  Returns a status code.
  */
 int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
 
