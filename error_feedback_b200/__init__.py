@@ -367,9 +367,10 @@ def topk_ef_path_info(ws, stream=None) -> dict:
 
 
 def topk_ef_phase_times(ws, stream=None) -> list:
-    """Diagnostic timestamps of the last compress call on ws (12 values, ns;
-    -1: step not run): select kernel phases, then the sampling block."""
-    ns = (ctypes.c_int64 * 12)()
+    """Diagnostic timestamps of the last compress call on ws (20 values, ns;
+    -1: step not run): select kernel phases, the sampling block, then the
+    streaming and select kernels' spans over all blocks."""
+    ns = (ctypes.c_int64 * 20)()
     _check(lib().topk_ef_phase_times(ws.data_ptr(), _stream(stream), ns), "topk_ef_phase_times")
     return [int(x) for x in ns]
 

@@ -62,13 +62,33 @@ struct Ctrl {
     uint32_t merge_bar[32]; // grid barrier counters, one per merge round
     uint32_t pad1[6];
     uint64_t t_phase[8];    // select kernel: globaltimer at each phase (block 0)
+    uint64_t t_span[8];     // globaltimer over all blocks (diagnostics): the first
+                            // block of a kernel stores ~t (atomicMax of the
+                            // complement), the last one t; SPAN_* below
 };
-static_assert(sizeof(Ctrl) == 256, "Ctrl layout");
+static_assert(sizeof(Ctrl) == 320, "Ctrl layout");
+
+// Slots of Ctrl::t_span.
+constexpr int SPAN_STREAM_FIRST = 0;   // streaming pass: first block past its wait on the setup
+constexpr int SPAN_STREAM_LAST = 1;    // streaming pass: last block done
+constexpr int SPAN_SELECT_FIRST = 2;   // select / threshold kernel: first block started
+constexpr int SPAN_SELECT_LAST = 3;    // select / threshold kernel: last block done
+constexpr int SPAN_GATHER_LAST = 4;    // its last block done gathering candidates
+constexpr int SPAN_BAR2_LAST = 5;      // its last block at the barrier after the entry lists
+constexpr int SPAN_OFFSET_LAST = 6;    // its last block with its output offset known
+constexpr int SPAN_START_LAST = 7;     // its last block started
 
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+__device__ __forceinline__ void span_first(Ctrl* c, int i) {
+    atomicMax(reinterpret_cast<unsigned long long*>(&c->t_span[i]), ~(unsigned long long)global_ns());
+}
+__device__ __forceinline__ void span_last(Ctrl* c, int i) {
+    atomicMax(reinterpret_cast<unsigned long long*>(&c->t_span[i]), (unsigned long long)global_ns());
 }
 
 // Every NaN gets the largest key (NaN payloads are implementation-defined:
@@ -157,8 +177,9 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t& epoch,
     if (threadIdx.x == 0) {
         epoch += 1;
         const uint32_t target = epoch * gridDim.x;
-        __threadfence();
-        atomicAdd(counter, 1u);
+        // release: the block's writes (ordered before by the block barrier)
+        // are visible to whoever acquires the count
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
         uint32_t it = 0;
         int ok = 1;
         while (ld_acquire_u32(counter) < target) {
@@ -167,9 +188,8 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t& epoch,
                 ok = 0;
                 break;
             }
-            __nanosleep(64);
+            if (it > 32) __nanosleep(64);   // poll back to back at first
         }
-        __threadfence();
         *s_flag = ok;
     }
     __syncthreads();

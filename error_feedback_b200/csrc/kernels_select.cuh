@@ -41,6 +41,8 @@ constexpr int EMIT_TILE = SEL_THREADS * EMIT_PER_THREAD;
 // Entry list of a prefiltered tensor: candidates in the bin of relative digit
 // 1 that holds the k-th key, as (block << 12) | relative digit 2.
 constexpr uint32_t ENT_PER = 4096;
+// Tiles of more than WT_THREAD candidates a warp gathers at once.
+constexpr int OVF_U = 4;
 
 struct Slot {
     int32_t l_first, l_last;
@@ -74,6 +76,8 @@ struct SelShared {
     uint32_t shift[SEG_MAX];
     FindResult fr;
     RelState rs[2];            // first and last segment of the block's range
+    RelState rs_early;         // one tensor, digit 1 built by the streaming pass
+    uint32_t top_bin;          // its candidates in the top relative bin (overflow)
     DigitState ds;
     DigitState fin[2];         // final thresholds of the first and last segment
     int flag;
@@ -134,16 +138,22 @@ __device__ void resolve_std(const uint32_t* h1, const uint32_t* h2, const uint32
 }
 
 // Relative digit 1 of a prefiltered tensor from its global histogram r1.
-__device__ RelState resolve_rel1(const uint32_t* r1, uint32_t k, SelShared& S) {
-    __syncthreads();
+// ... from the histogram already in S.stage.
+__device__ RelState rel1_from_stage(uint32_t k, SelShared& S) {
     if (k == 0) return RelState{0u, 0u, 0u, 0u};
-    stage_words(S.stage, r1, REL_BINS, REL_BINS);
-    __syncthreads();
     block_find_bin(S.stage, REL_BINS, k, S.red, &S.fr);
     const RelState r{S.fr.bin, k - S.fr.above, S.fr.cnt,
                      (S.fr.ok && S.fr.bin != REL_BINS - 1) ? 1u : 0u};
     __syncthreads();
     return r;
+}
+
+__device__ RelState resolve_rel1(const uint32_t* r1, uint32_t k, SelShared& S) {
+    __syncthreads();
+    if (k == 0) return RelState{0u, 0u, 0u, 0u};
+    stage_words(S.stage, r1, REL_BINS, REL_BINS);
+    __syncthreads();
+    return rel1_from_stage(k, S);
 }
 
 // T (prefix) and the tie quota (rem) from the relative digit-2 histogram h2
@@ -316,33 +326,66 @@ __device__ __forceinline__ bool in_class(uint32_t key, int d, uint32_t prefix) {
 __device__ __forceinline__ void mark_phase(Ctrl* ctrl, int i) {
     if (blockIdx.x == 0 && threadIdx.x == 0) ctrl->t_phase[i] = global_ns();
 }
+// The same phase, latest over all blocks.
+__device__ __forceinline__ void mark_last(Ctrl* ctrl, int slot) {
+    if (threadIdx.x == 0) span_last(ctrl, slot);
+}
+
+// First start and last end over the blocks of a select-type kernel (thread 0
+// of each block; its end is stamped on every return path).
+struct BlockSpan {
+    Ctrl* c;
+    __device__ explicit BlockSpan(Ctrl* ctrl) : c(ctrl) {
+        if (threadIdx.x == 0) {
+            span_first(c, SPAN_SELECT_FIRST);
+            span_last(c, SPAN_START_LAST);
+        }
+    }
+    __device__ ~BlockSpan() {
+        if (threadIdx.x == 0) span_last(c, SPAN_SELECT_LAST);
+    }
+};
 
 // Output offset of a block inside segment l from the blocks before it: the
 // (gt, eq) counts of the run of earlier blocks whose ranges continue l (their
-// slots), summed by warp 0.  Result in S.pre[0..1].
+// slots), summed by warp 0, which loads the slots of 128 blocks at a time.
+// Result in S.pre[0..1].
 __device__ void chain_prefix(const SelCommon& cm, int c, int l, SelShared& S) {
+    constexpr int U = 4;
     if (threadIdx.x < 32) {
+        const uint32_t lane = lane_id();
         uint32_t pg = 0, pe = 0;
-        int cc = c - 1;
-        for (;;) {
-            const int j = cc - (int)lane_id();
-            bool match = false, cont = false;
-            uint32_t g = 0, e = 0;
-            if (j >= 0) {
-                const Slot sl = cm.slots[j];
-                match = sl.l_last == l;
-                cont = match && sl.l_first == l;
-                g = sl.gt_last;
-                e = sl.eq_last;
+        bool done = false;
+        for (int c0 = c - 1; !done; c0 -= 32 * U) {
+            int lf[U], ll[U];
+            uint32_t g[U], e[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int j = c0 - 32 * u - (int)lane;
+                lf[u] = ll[u] = -1;
+                g[u] = e[u] = 0;
+                if (j >= 0) {
+                    const uint4* q = reinterpret_cast<const uint4*>(cm.slots + j);
+                    const uint4 a = q[0], b = q[1];
+                    lf[u] = (int)a.x;
+                    ll[u] = (int)a.y;
+                    g[u] = b.x;    // gt_last
+                    e[u] = b.y;    // eq_last
+                }
             }
-            const uint32_t contm = __ballot_sync(0xFFFFFFFFu, cont);
-            const uint32_t matchm = __ballot_sync(0xFFFFFFFFu, match);
-            const uint32_t run = (contm == 0xFFFFFFFFu) ? 32u : (uint32_t)(__ffs(~contm) - 1);
-            const bool take = lane_id() < run || (lane_id() == run && ((matchm >> run) & 1u));
-            pg += warp_sum(take ? g : 0u);
-            pe += warp_sum(take ? e : 0u);
-            if (run < 32) break;
-            cc -= 32;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (done) continue;
+                const bool match = ll[u] == l;
+                const bool cont = match && lf[u] == l;
+                const uint32_t contm = __ballot_sync(0xFFFFFFFFu, cont);
+                const uint32_t matchm = __ballot_sync(0xFFFFFFFFu, match);
+                const uint32_t run = (contm == 0xFFFFFFFFu) ? 32u : (uint32_t)(__ffs(~contm) - 1);
+                const bool take = lane < run || (lane == run && ((matchm >> run) & 1u));
+                pg += warp_sum(take ? g[u] : 0u);
+                pe += warp_sum(take ? e[u] : 0u);
+                if (run < 32) done = true;
+            }
         }
         if (threadIdx.x == 0) {
             S.pre[0] = pg;
@@ -421,21 +464,32 @@ struct TileCands {
     float v[WT_THREAD];
 };
 
-__device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, uint32_t cnt,
-                                            TileCands& t) {
+// The offsets: their loads do not depend on the count (the slots past it
+// hold stale data, masked by load_values), so they are issued together with
+// the load of the count.
+__device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, TileCands& t) {
     const uint4* p4 = reinterpret_cast<const uint4*>(src.wt_off + (size_t)w * WT_CAP);
-    const uint4 a = p4[0];
+    const uint4 a = p4[0], b = p4[1];
     t.o[0] = a.x & 0xFFFFu; t.o[1] = a.x >> 16; t.o[2] = a.y & 0xFFFFu; t.o[3] = a.y >> 16;
     t.o[4] = a.z & 0xFFFFu; t.o[5] = a.z >> 16; t.o[6] = a.w & 0xFFFFu; t.o[7] = a.w >> 16;
-    uint4 b = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-    if (cnt > 8) b = p4[1];
     t.o[8] = b.x & 0xFFFFu; t.o[9] = b.x >> 16; t.o[10] = b.y & 0xFFFFu; t.o[11] = b.y >> 16;
     t.o[12] = b.z & 0xFFFFu; t.o[13] = b.z >> 16; t.o[14] = b.w & 0xFFFFu; t.o[15] = b.w >> 16;
+}
+
+// The values of the first cnt slots (cnt <= WT_THREAD; none for a larger
+// tile, which a warp gathers), and the masking of the other slots.
+__device__ __forceinline__ void load_values(const CompressSrc& src, uint32_t w, uint32_t cnt,
+                                            TileCands& t) {
     const int64_t base = (int64_t)w * WT;
+    const uint32_t c = cnt <= (uint32_t)WT_THREAD ? cnt : 0u;
 #pragma unroll
     for (int i = 0; i < WT_THREAD; ++i) {
-        if ((uint32_t)i >= cnt) t.o[i] = 0xFFFFu;
-        t.v[i] = (uint32_t)i < cnt ? src.resid[base + t.o[i]] : 0.f;
+        if ((uint32_t)i < c) {
+            t.v[i] = src.resid[base + t.o[i]];
+        } else {
+            t.o[i] = 0xFFFFu;
+            t.v[i] = 0.f;
+        }
     }
 }
 
@@ -447,7 +501,7 @@ __device__ __forceinline__ void load_staged(const CompressSrc& src, uint32_t w, 
 // candidate is sent, so its residual becomes +0.0f, and there is no
 // histogram.
 template <int C, bool kThr>
-__device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelShared& S,
+__device__ __forceinline__ void store_ranked(const CompressSrc& src, SelShared& S,
                                              uint32_t w, uint64_t pos, uint32_t cnt,
                                              const TileCands& t, uint32_t* s_r1, int lc) {
     const int64_t base = (int64_t)w * WT;
@@ -468,53 +522,46 @@ __device__ __forceinline__ void store_ranked(const CompressSrc& src, const SelSh
     }
 }
 
-// Output offset of block c's candidates: the sum of the counts the blocks
-// before it published (count + 1; 0 = not yet), read by warp 0.  Every block
-// publishes before any heavy work and all blocks are resident, so the wait
-// is short; it is bounded all the same.
-__device__ uint64_t look_back(const uint64_t* agg, int c, uint32_t* status, SelShared& S) {
-    if (threadIdx.x < 32) {
-        uint64_t sum = 0;
-        for (int j = (int)lane_id(); j < c; j += 32) {
-            uint64_t v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
-            uint32_t it = 0;
-            while (v == 0) {
-                if (++it > SPIN_LIMIT) {
-                    atomicOr(status, ST_TIMEOUT);
-                    break;
-                }
-                __nanosleep(32);
-                v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
-            }
-            sum += v ? v - 1 : 0;
+// Published count (+1) of block j, waited for: every block publishes before
+// any heavy work and all blocks are resident, so the wait is short; it is
+// bounded all the same.
+__device__ __forceinline__ uint64_t agg_wait(const uint64_t* agg, int j, uint64_t v,
+                                             uint32_t* status) {
+    uint32_t it = 0;
+    while (v == 0) {
+        if (++it > SPIN_LIMIT) {
+            atomicOr(status, ST_TIMEOUT);
+            break;
         }
-        sum = warp_sum(sum);
-        if (threadIdx.x == 0) S.before = sum;
+        if (it > 32) __nanosleep(32);
+        v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
     }
-    __syncthreads();
-    return S.before;
+    return v ? v - 1 : 0;
 }
 
-// Output offset of block c and the total of all blocks (warp 0 reads every
-// published count; all blocks publish before any heavy work, so the wait is
-// short; bounded all the same).  Results in S.before and S.total.
-__device__ void look_all(const uint64_t* agg, int c, uint32_t* status, SelShared& S) {
+// Candidates of blocks [0, c) (S.before) and, with `all`, of every block
+// (S.total), summed by warp 0 from the published counts.  The loads of a
+// round of 8 per lane are issued together.
+template <bool all>
+__device__ void look_counts(const uint64_t* agg, int c, uint32_t* status, SelShared& S) {
     if (threadIdx.x < 32) {
+        const int G = all ? (int)gridDim.x : c;
         uint64_t before = 0, total = 0;
-        for (int j = (int)lane_id(); j < (int)gridDim.x; j += 32) {
-            uint64_t v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
-            uint32_t it = 0;
-            while (v == 0) {
-                if (++it > SPIN_LIMIT) {
-                    atomicOr(status, ST_TIMEOUT);
-                    break;
-                }
-                __nanosleep(32);
-                v = *reinterpret_cast<const volatile uint64_t*>(agg + j);
+        for (int j0 = 0; j0 < G; j0 += 32 * 8) {
+            uint64_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + 32 * u + (int)lane_id();
+                v[u] = j < G ? *reinterpret_cast<const volatile uint64_t*>(agg + j) : 1u;
             }
-            const uint64_t cnt = v ? v - 1 : 0;
-            total += cnt;
-            if (j < c) before += cnt;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + 32 * u + (int)lane_id();
+                if (j >= G) continue;
+                const uint64_t cnt = agg_wait(agg, j, v[u], status);
+                total += cnt;
+                if (j < c) before += cnt;
+            }
         }
         before = warp_sum(before);
         total = warp_sum(total);
@@ -527,20 +574,19 @@ __device__ void look_all(const uint64_t* agg, int c, uint32_t* status, SelShared
 }
 
 // Gather a warp tile with WT_THREAD < cnt <= WT_CAP staged candidates (one
-// warp): lane i takes offset i, ranks it among the others by shuffles and
-// reads its value back from the residual.
+// warp), its offset o and value v already loaded by lane i < cnt (staged
+// slot i; 0xFFFF elsewhere): each lane ranks its offset among the others by
+// shuffles and writes its candidate.
 template <bool kThr>
-__device__ void gather_warp_staged(const CompressSrc& src, const SelShared& S, uint32_t w,
-                                   uint64_t pos, uint32_t cnt, uint32_t* s_r1, int lc) {
+__device__ __forceinline__ void store_warp_staged(const CompressSrc& src, SelShared& S,
+                                                  uint32_t w, uint64_t pos, uint32_t cnt,
+                                                  uint32_t o, float v, uint32_t* s_r1, int lc) {
     const uint32_t lane = lane_id();
-    const int64_t base = (int64_t)w * WT;
-    const uint32_t o = lane < cnt ? (uint32_t)src.wt_off[(size_t)w * WT_CAP + lane] : 0xFFFFu;
     uint32_t rank = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) rank += __shfl_sync(0xFFFFFFFFu, o, i) < o;
     if (lane < cnt) {
-        const int64_t e = base + o;
-        const float v = src.resid[e];
+        const int64_t e = (int64_t)w * WT + o;
         const uint64_t q = pos + rank;
         if (q < src.cap) {
             src.cand_idx[q] = (uint32_t)e;
@@ -551,17 +597,88 @@ __device__ void gather_warp_staged(const CompressSrc& src, const SelShared& S, u
     }
 }
 
+__device__ __forceinline__ float f4_get(const float4& v, int t) {
+    return t == 0 ? v.x : (t == 1 ? v.y : (t == 2 ? v.z : v.w));
+}
+
 // Gather a warp tile with more than WT_CAP candidates (one warp): rescan it
-// from the residual (which holds acc) with the streaming pass's test.  The
-// 32 coalesced loads of the tile (element base + 32 u + lane) are issued at
-// once; one ballot per load gives the positions in index order.
+// from the residual (which holds acc) with the streaming pass's test.  A
+// full tile with a 16-byte aligned base is read as 8 float4 per lane (lane
+// holds elements 128 j + 4 lane + t, so within each j the candidates are in
+// index order lane by lane: one warp scan places them); any other tile as 32
+// coalesced scalar loads (element 32 u + lane) with one ballot each.  All the
+// loads of a tile are issued before the first is used.  Out of line: it runs
+// for dense tiles only and keeps its registers to itself.
+// What the rescan needs of CompressSrc, passed by value (a reference would
+// make the caller keep a copy of the whole source in local memory).
+struct RescanArgs {
+    float* resid;
+    int64_t N;
+    uint32_t* cand_idx;
+    float* cand_val;
+    uint64_t cap;
+    uint32_t* hist;
+    int32_t T;
+    int32_t r1_done;
+    __device__ explicit RescanArgs(const CompressSrc& s)
+        : resid(s.resid), N(s.N), cand_idx(s.cand_idx), cand_val(s.cand_val), cap(s.cap),
+          hist(s.hist), T(s.T), r1_done(s.r1_done) {}
+    __device__ void r1_add(const SelShared& S, int l, float v, uint32_t* s_r1) const {
+        const uint32_t bin = rel_bin(key_of(v), S.T0[l], S.shift[l]);
+        if (s_r1) atomicAdd(&s_r1[bin], 1u);
+        else atomicAdd(hist + (size_t)l * CHIST_WORDS + CH_R1 + bin, 1u);
+    }
+};
+
 template <bool kThr>
-__device__ void gather_rescan(const CompressSrc& src, const SelShared& S, uint32_t w,
-                              uint64_t pos, uint32_t* s_r1, int lc) {
+__device__ __noinline__ void gather_rescan(const RescanArgs src, SelShared& S, uint32_t w,
+                                           uint64_t pos, uint32_t* s_r1, int lc) {
     const uint32_t lane = lane_id();
     const int T = src.T;
     const int64_t base = (int64_t)w * WT;
     const int64_t tend = min(base + (int64_t)WT, src.N);
+    const float* tile = src.resid + base;
+    if (tend - base == WT && (reinterpret_cast<uintptr_t>(tile) & 15u) == 0) {
+        const float4* t4 = reinterpret_cast<const float4*>(tile) + lane;
+        float4 v4[WT_VECS];
+#pragma unroll
+        for (int j = 0; j < WT_VECS; ++j) v4[j] = t4[32 * j];
+        int l = lc;
+        if (!s_r1) l = seg_of(S.seg, T, base + 4 * (int64_t)lane);
+#pragma unroll
+        for (int j = 0; j < WT_VECS; ++j) {
+            const int64_t e0 = base + 128 * j + 4 * (int64_t)lane;
+            const int lj = l;
+            uint32_t f = 0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if (!s_r1)
+                    while (l < T - 1 && S.seg[l + 1] <= e0 + t) ++l;
+                f |= (uint32_t)(key_of(f4_get(v4[j], t)) >= S.T0[l]) << t;
+            }
+            const uint32_t c = (uint32_t)__popc(f);
+            const uint32_t incl = warp_incl_scan(c);
+            uint64_t q = pos + incl - c;
+            int l2 = lj;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if (!s_r1)
+                    while (l2 < T - 1 && S.seg[l2 + 1] <= e0 + t) ++l2;
+                if ((f >> t) & 1u) {
+                    const float a = f4_get(v4[j], t);
+                    if (q < src.cap) {
+                        src.cand_idx[q] = (uint32_t)(e0 + t);
+                        src.cand_val[q] = a;
+                        if (kThr) src.resid[e0 + t] = 0.0f;
+                    }
+                    if (!kThr && !src.r1_done) src.r1_add(S, l2, a, s_r1);
+                    ++q;
+                }
+            }
+            pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        return;
+    }
     float v[32];
 #pragma unroll
     for (int u = 0; u < 32; ++u) {
@@ -589,7 +706,7 @@ __device__ void gather_rescan(const CompressSrc& src, const SelShared& S, uint32
                 src.cand_val[q] = v[u];
                 if (kThr) src.resid[e] = 0.0f;
             }
-            if (!kThr && !src.r1_done) r1_add(src, S, l, v[u], s_r1);
+            if (!kThr && !src.r1_done) src.r1_add(S, l, v[u], s_r1);
         }
         pos += __popc(m);
     }
@@ -627,53 +744,86 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
     const int T = src.T;
     uint32_t* status = &cm.ctrl->status;
     int64_t* s_off = S.seg;
+    const uint32_t W = src.num_wt;
+    const uint32_t per = (W + G - 1) / G;
+    const uint32_t w0 = min((uint32_t)c * per, W), w1 = min(w0 + per, W);
+    // the first round's tile of this thread, loaded before anything else
+    uint32_t cnt = 0;
+    TileCands tc;
+    if (w0 + tid < w1) {
+        cnt = src.wt_count[w0 + tid];
+        load_staged(src, w0 + tid, tc);
+    }
+    // one tensor whose relative digit 1 the streaming pass built: that
+    // histogram too (REL_BINS words, two 16-byte words per thread)
+    static_assert(REL_BINS == 8 * SEL_THREADS, "digit-1 histogram load");
+    const bool early = !kThr && src.r1_done;
+    uint4 r1v[2];
+    if (early) {
+        const uint4* h4 = reinterpret_cast<const uint4*>(src.h(0, CH_R1));
+        r1v[0] = h4[tid];
+        r1v[1] = h4[tid + SEL_THREADS];
+    }
     for (int l = tid; l < T; l += blockDim.x) {
         s_off[l] = src.meta[l].off;
         S.T0[l] = src.meta[l].T0;
         S.shift[l] = src.meta[l].shift;
     }
     if (tid == 0) s_off[T] = src.N;
-    const uint32_t W = src.num_wt;
-    const uint32_t per = (W + G - 1) / G;
-    const uint32_t w0 = min((uint32_t)c * per, W), w1 = min(w0 + per, W);
-
+    // one round: the block's count is the first scan's total, published
+    // there; otherwise it is summed and published first
+    const bool single = w1 - w0 <= blockDim.x;
     uint32_t mine = 0;
-    for (uint32_t w = w0 + tid; w < w1; w += blockDim.x) mine += src.wt_count[w];
-    mine = block_sum(mine, S.red);
-    if (tid == 0) {
-        __threadfence();
-        *reinterpret_cast<volatile uint64_t*>(src.agg + c) = (uint64_t)mine + 1;
+    if (!single) {
+        mine = cnt;
+        for (uint32_t w = w0 + tid + blockDim.x; w < w1; w += blockDim.x) mine += src.wt_count[w];
+        mine = block_sum(mine, S.red);
+        if (tid == 0) *reinterpret_cast<volatile uint64_t*>(src.agg + c) = (uint64_t)mine + 1;
     }
 
     // relative digit 1 in shared memory when the whole chunk is in one tensor
     const int64_t e0 = (int64_t)w0 * WT, e1 = min((int64_t)w1 * WT, src.N);
+    __syncthreads();
     const int lc = w0 < w1 ? seg_of(s_off, T, e0) : 0;
     const bool one = !kThr && !src.r1_done && w0 < w1 && seg_of(s_off, T, e1 - 1) == lc;
     uint32_t* s_r1 = one ? S.stage : nullptr;
     if (one)
         for (int i = tid; i < REL_BINS; i += blockDim.x) S.stage[i] = 0;
-    // tiles with more than WT_THREAD candidates of a piece: (tile, position)
+    // tiles with more than WT_THREAD candidates of a piece: tile, count
+    // (SEL_THREADS words further) and output position
+    static_assert(2 * SEL_THREADS <= D1_BINS, "overflow tile list");
     uint32_t* s_ovf_w = S.h1;
     uint64_t before = 0, run = 0;
     bool have_before = false;
     for (uint32_t pw = w0; pw < w1 || !have_before; pw += blockDim.x) {
         const uint32_t w = pw + tid;
-        const uint32_t cnt = w < w1 ? src.wt_count[w] : 0u;
         if (tid == 0) S.flag = 0;
         uint32_t piece;
         const uint32_t ex = block_excl_scan(cnt, S.red, &piece);
-        TileCands tc;
-        const bool staged = cnt > 0 && cnt <= (uint32_t)WT_THREAD;
-        if (staged) load_staged(src, w, cnt, tc);
+        if (single) {
+            mine = piece;
+            if (tid == 0) *reinterpret_cast<volatile uint64_t*>(src.agg + c) = (uint64_t)mine + 1;
+        }
+        load_values(src, w, cnt, tc);
         if (!have_before) {
-            if (src.r1_done) {
-                look_all(src.agg, c, status, S);
-                before = S.before;
-            } else {
-                before = look_back(src.agg, c, status, S);
+            // resolved while the other blocks publish their counts
+            if (early) {
+                uint4* s4 = reinterpret_cast<uint4*>(S.stage);
+                s4[tid] = r1v[0];
+                s4[tid + SEL_THREADS] = r1v[1];
+                __syncthreads();
+                const RelState r = rel1_from_stage(src.meta[0].k, S);
+                if (tid == 0) {
+                    S.rs_early = r;
+                    S.top_bin = S.stage[REL_BINS - 1];
+                }
             }
+            if (src.r1_done) look_counts<true>(src.agg, c, status, S);
+            else look_counts<false>(src.agg, c, status, S);
+            before = S.before;
             have_before = true;
             mark_phase(cm.ctrl, 4);
+            mark_last(cm.ctrl, SPAN_OFFSET_LAST);
         }
         const uint64_t pos = before + run + ex;
         if (w < w1 && T > 1) {
@@ -682,24 +832,57 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
             for (int l = max(1, lower_bound_off(s_off, T, base)); l < T && s_off[l] < tend; ++l)
                 src.cand_start[l] = (int64_t)(pos + tile_count_below(src, S, w, cnt, s_off[l]));
         }
-        if (cnt > (uint32_t)WT_THREAD) {
+        if (pos >= src.cap) {
+            // past the capacity: nothing of this tile is written (a compress
+            // call then falls back to the rescan; the hard-threshold step
+            // sends only the first cap)
+        } else if (cnt > (uint32_t)WT_THREAD) {
             const uint32_t slot = atomicAdd(reinterpret_cast<uint32_t*>(&S.flag), 1u);
             s_ovf_w[slot] = w;
+            s_ovf_w[SEL_THREADS + slot] = cnt;
             S.ovf_pos[slot] = pos;
         } else if (cnt > 4) {
             store_ranked<WT_THREAD, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         } else if (cnt > 0) {
             store_ranked<4, kThr>(src, S, w, pos, cnt, tc, s_r1, lc);
         }
-        __syncthreads();
-        const uint32_t novf = (uint32_t)S.flag;
-        for (uint32_t i = warp; i < novf; i += nwarps) {
-            const uint32_t wo = s_ovf_w[i];
-            if (src.wt_count[wo] <= (uint32_t)WT_CAP)
-                gather_warp_staged<kThr>(src, S, wo, S.ovf_pos[i], src.wt_count[wo], s_r1, lc);
-            else
-                gather_rescan<kThr>(src, S, wo, S.ovf_pos[i], s_r1, lc);
+        // the next round's tile
+        cnt = 0;
+        if (w + blockDim.x < w1) {
+            cnt = src.wt_count[w + blockDim.x];
+            load_staged(src, w + blockDim.x, tc);
         }
+        __syncthreads();
+        // tiles of more than WT_THREAD candidates, a warp each; the loads of
+        // OVF_U staged tiles of a warp are issued together
+        const uint32_t novf = (uint32_t)S.flag;
+        for (uint32_t i0 = warp; i0 < novf; i0 += nwarps * OVF_U) {
+            uint32_t wo[OVF_U], cn[OVF_U], o[OVF_U];
+            float v[OVF_U];
+#pragma unroll
+            for (int u = 0; u < OVF_U; ++u) {
+                const uint32_t i = i0 + u * nwarps;
+                wo[u] = i < novf ? s_ovf_w[i] : 0u;
+                cn[u] = i < novf ? s_ovf_w[SEL_THREADS + i] : 0u;
+                const bool st = cn[u] <= (uint32_t)WT_CAP && lane_id() < cn[u];
+                o[u] = st ? (uint32_t)src.wt_off[(size_t)wo[u] * WT_CAP + lane_id()] : 0xFFFFu;
+            }
+#pragma unroll
+            for (int u = 0; u < OVF_U; ++u) {
+                const bool st = cn[u] <= (uint32_t)WT_CAP && lane_id() < cn[u];
+                v[u] = st ? src.resid[(int64_t)wo[u] * WT + o[u]] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < OVF_U; ++u) {
+                const uint32_t i = i0 + u * nwarps;
+                if (i < novf && cn[u] <= (uint32_t)WT_CAP)
+                    store_warp_staged<kThr>(src, S, wo[u], S.ovf_pos[i], cn[u], o[u], v[u], s_r1, lc);
+            }
+        }
+        // more than WT_CAP: rescanned
+        for (uint32_t i = warp; i < novf; i += nwarps)
+            if (s_ovf_w[SEL_THREADS + i] > (uint32_t)WT_CAP)
+                gather_rescan<kThr>(RescanArgs(src), S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
         __syncthreads();
         run += piece;
     }
@@ -717,6 +900,7 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
             if (S.stage[i]) atomicAdd(&g[i], S.stage[i]);
     }
     mark_phase(cm.ctrl, 5);
+    mark_last(cm.ctrl, SPAN_GATHER_LAST);
 }
 
 // The gather phase, one grid barrier, and the decision every block takes
@@ -734,7 +918,8 @@ __device__ bool compress_gather(CompressSrc& src, const SelCommon& cm, uint32_t&
         // one tensor, relative digit 1 built by the streaming pass and the
         // total known from the look-all: no barrier needed to decide
         total = S.total;
-        bad = (total < (uint64_t)src.meta[0].k) || src.rel_overflow(0);
+        const uint32_t k = src.meta[0].k;
+        bad = (total < (uint64_t)k) || (k > 0 && S.top_bin >= k);
         mark_phase(cm.ctrl, 1);
     } else {
         if (!grid_barrier(cm.bar, epoch, &cm.ctrl->status, &S.flag)) return false;
@@ -765,6 +950,7 @@ __global__ void __launch_bounds__(SEL_THREADS)
 threshold_kernel(CompressSrc src, SelCommon cm, int64_t* out_count) {
     __shared__ SelShared S;
     mark_phase(cm.ctrl, 0);
+    const BlockSpan block_span(cm.ctrl);
     uint64_t my0, my1;
     gather_phase<true>(src, cm, S, my0, my1);
     if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
@@ -886,8 +1072,11 @@ __device__ bool local_small(const CompressSrc& src, int l, int64_t a, int64_t b,
 }
 
 // Selection and emission on the dense candidate list.  The block's range
-// [a0, a1) is what it gathered.  A tensor that lies wholly inside the range
-// is finished here alone.  For the (at most two) tensors that cross the
+// [a0, a1) is what it gathered.  A small tensor (at most EMIT_TILE
+// candidates) is selected from registers by one block after the barrier,
+// block l mod G for tensor l, so that a range holding many of them does not
+// hold up the grid.  A larger tensor that lies wholly inside the range is
+// finished here alone.  For the (at most two) tensors that cross the
 // range's ends: count the candidates above the k-th key's digit-1 bin (slot)
 // and put the candidates in the bin on the tensor's entry list; after a
 // barrier every block reads T, the tie quota and the entries of the blocks
@@ -922,12 +1111,10 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
         const int64_t b = min((int64_t)a1, S.seg[l + 1]);
         if (a >= b) continue;
         const uint32_t k = src.meta[l].k;
+        // a small tensor is selected by one block after the barrier
+        if (S.seg[l + 1] - S.seg[l] <= (int64_t)EMIT_TILE) continue;
         const bool local = S.seg[l] >= (int64_t)a0 && S.seg[l + 1] <= (int64_t)a1;
-        if (local && b - a <= (int64_t)EMIT_TILE) {
-            if (!local_small(src, l, a, b, S) && tid == 0) atomicOr(status, ST_INCONSISTENT);
-            continue;
-        }
-        const RelState rs = resolve_rel1(src.h(l, CH_R1), k, S);
+        const RelState rs = src.r1_done ? S.rs_early : resolve_rel1(src.h(l, CH_R1), k, S);
         if (!rs.ok) {
             if (k && tid == 0) atomicOr(status, ST_INCONSISTENT);
             continue;
@@ -975,11 +1162,20 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
         sl.pad[0] = sl.pad[1] = 0;
         cm.slots[c] = sl;
     }
+    mark_last(cm.ctrl, SPAN_BAR2_LAST);
     if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
     mark_phase(cm.ctrl, 2);
     const bool r2p = *reinterpret_cast<volatile uint32_t*>(&cm.ctrl->r2_path) != 0;
 
-    // T and the tie quota of the crossing tensors
+    // T and the tie quota of the crossing tensors.  The entry words are
+    // loaded together with their count (slots past it hold stale words and
+    // are dropped); the first tensor's stay in registers for the count of
+    // the entries of earlier blocks, whose slots warp 0 reads meanwhile.
+    constexpr int EPT = (int)ENT_PER / SEL_THREADS;
+    uint32_t ev0[EPT];
+#pragma unroll
+    for (int u = 0; u < EPT; ++u) ev0[u] = DEAD;
+    const bool chain0 = cross[0] && max((int64_t)a0, S.seg[l_first]) > S.seg[l_first];
     DigitState fin[2];
 #pragma unroll
     for (int side = 0; side < 2; ++side) {
@@ -987,12 +1183,26 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
         if (!cross[side]) continue;
         const int l = side == 0 ? l_first : l_last;
         const RelState rs = S.rs[side];
-        zero_stage(S);
         if (rs.cnt <= ENT_PER) {
-            const uint32_t E = min(*reinterpret_cast<volatile uint32_t*>(src.ent_cnt + l), ENT_PER);
             const uint32_t* el = src.ent + (size_t)l * ENT_PER;
-            for (uint32_t i = tid; i < E; i += blockDim.x) atomicAdd(&S.stage[el[i] & 4095u], 1u);
+            uint32_t ev[EPT];
+            const uint32_t E = min(*reinterpret_cast<volatile uint32_t*>(src.ent_cnt + l), ENT_PER);
+#pragma unroll
+            for (int u = 0; u < EPT; ++u) ev[u] = el[tid + u * SEL_THREADS];
+#pragma unroll
+            for (int u = 0; u < EPT; ++u)
+                if ((uint32_t)(tid + u * SEL_THREADS) >= E) ev[u] = DEAD;
+            if (side == 0) {
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) ev0[u] = ev[u];
+                if (chain0 && !r2p) chain_prefix(cm, c, l, S);
+            }
+            zero_stage(S);
+#pragma unroll
+            for (int u = 0; u < EPT; ++u)
+                if (ev[u] != DEAD) atomicAdd(&S.stage[ev[u] & 4095u], 1u);
         } else {
+            zero_stage(S);
             stage_words(S.stage, src.h(l, CH_R2), REL_BINS, REL_BINS);
         }
         __syncthreads();
@@ -1043,8 +1253,8 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
         const int64_t a = max((int64_t)a0, S.seg[l]);
         const int64_t b = min((int64_t)a1, S.seg[l + 1]);
         uint32_t pg = 0, pe = 0;
-        if (side == 0 && a > S.seg[l]) {
-            chain_prefix(cm, c, l, S);
+        if (side == 0 && chain0) {
+            if (r2p) chain_prefix(cm, c, l, S);   // the slots now hold exact counts
             pg = S.pre[0];
             pe = S.pre[1];
             __syncthreads();
@@ -1052,12 +1262,11 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
                 // candidates of the k-th key's bin held by earlier blocks
                 const RelState rs = S.rs[0];
                 const uint32_t t = fin[0].prefix - S.T0[l] - (rs.b1 << S.shift[l]);
-                const uint32_t E = min(src.ent_cnt[l], ENT_PER);
-                const uint32_t* el = src.ent + (size_t)l * ENT_PER;
                 uint32_t g = 0, e = 0;
-                for (uint32_t i = tid; i < E; i += blockDim.x) {
-                    const uint32_t v = el[i];
-                    if ((int)(v >> 12) < c) {
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) {
+                    const uint32_t v = ev0[u];
+                    if (v != DEAD && (int)(v >> 12) < c) {
                         g += (v & 4095u) > t;
                         e += (v & 4095u) == t;
                     }
@@ -1067,6 +1276,13 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
             }
         }
         emit_range(src, l, a, b, fin[side].prefix, fin[side].rem, src.meta[l].k, pg, pe, S);
+    }
+    // small tensors (at most EMIT_TILE candidates), tensor l by block l mod G:
+    // their candidates are all written, wherever they were gathered
+    for (int l = c; l < T; l += (int)gridDim.x) {
+        const int64_t a = S.seg[l], b = S.seg[l + 1];
+        if (b > a && b - a <= (int64_t)EMIT_TILE && !local_small(src, l, a, b, S) && tid == 0)
+            atomicOr(status, ST_INCONSISTENT);
     }
     mark_phase(cm.ctrl, 7);
 }
@@ -1083,6 +1299,7 @@ select_kernel(Src src, SelCommon cm) {
     uint32_t epoch = 0;
     uint32_t* status = &cm.ctrl->status;
     mark_phase(cm.ctrl, 0);
+    const BlockSpan block_span(cm.ctrl);
 
     int first_digit;
     if constexpr (std::is_same<Src, CompressSrc>::value) {

@@ -102,24 +102,50 @@ __device__ __noinline__ uint32_t stream_tile_general(const StreamParams& p, Stre
 // them, their offsets in the tile (lane-major, so not in index order; the
 // select kernel sorts each tile's few offsets and reads the values back from
 // the residual, which now holds acc).  Bit 4j + v of a lane's flags is offset
-// 128 j + 4 lane + v.
-__device__ __forceinline__ void stream_tile_stage(const StreamParams& p, uint32_t w, uint32_t flags) {
+// 128 j + 4 lane + v.  With kRegs and hist, each candidate is also counted in
+// the relative digit-1 histogram s_r1 (its acc in the caller's registers:
+// element 128 j + 4 lane + v in rv[j]) in the same walk over the flags.
+template <bool kRegs>
+__device__ __forceinline__ void stream_tile_stage(const StreamParams& p, uint32_t w, uint32_t flags,
+                                                  const float4* rv, bool hist, uint32_t* s_r1,
+                                                  uint32_t T0, uint32_t sh) {
     const uint32_t lane = lane_id();
     const uint32_t pc = (uint32_t)__popc(flags);
     const uint32_t incl = warp_incl_scan(pc);
     if (lane == 31) p.wt_count[w] = incl;
     uint32_t pos = incl - pc;
     uint16_t* dst = p.wt_off + (size_t)w * WT_CAP;
-    while (flags && pos < (uint32_t)WT_CAP) {
-        const uint32_t b = (uint32_t)(__ffs(flags) - 1);
-        flags &= flags - 1;
-        dst[pos++] = (uint16_t)(128u * (b >> 2) + 4u * lane + (b & 3u));
+    if (kRegs && hist) {
+#pragma unroll
+        for (int j = 0; j < WT_VECS; ++j) {
+            const uint32_t f4 = (flags >> (4 * j)) & 0xFu;
+            if (f4 == 0) continue;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                if ((f4 >> v) & 1u) {
+                    if (pos < (uint32_t)WT_CAP) dst[pos] = (uint16_t)(128u * j + 4u * lane + v);
+                    ++pos;
+                    const float a = v == 0 ? rv[j].x : (v == 1 ? rv[j].y : (v == 2 ? rv[j].z : rv[j].w));
+                    atomicAdd(&s_r1[stream_rel_bin(a, T0, sh)], 1u);
+                }
+            }
+        }
+    } else {
+        while (flags && pos < (uint32_t)WT_CAP) {
+            const uint32_t b = (uint32_t)(__ffs(flags) - 1);
+            flags &= flags - 1;
+            dst[pos++] = (uint16_t)(128u * (b >> 2) + 4u * lane + (b & 3u));
+        }
     }
 }
 
+template <bool kRegs>
 __device__ __forceinline__ void stream_tile_record(const StreamParams& p, uint32_t w,
-                                                   uint32_t flags) {
-    if (__any_sync(0xFFFFFFFFu, flags != 0)) stream_tile_stage(p, w, flags);
+                                                   uint32_t flags, const float4* rv,
+                                                   bool hist = false, uint32_t* s_r1 = nullptr,
+                                                   uint32_t T0 = 0, uint32_t sh = 0) {
+    if (__any_sync(0xFFFFFFFFu, flags != 0))
+        stream_tile_stage<kRegs>(p, w, flags, rv, hist, s_r1, T0, sh);
     else if (lane_id() == 0) p.wt_count[w] = 0;
 }
 
@@ -157,6 +183,7 @@ stream_kernel(const __grid_constant__ StreamParams p) {
         }
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");   // setup_kernel's results
+    if (tid == 0) span_first(p.ctrl, SPAN_STREAM_FIRST);
     const uint32_t lane = lane_id();
     const int T = p.T;
     const bool flat = (T == 1);
@@ -222,28 +249,18 @@ stream_kernel(const __grid_constant__ StreamParams p) {
                 flags |= (uint32_t)((__float_as_uint(a.w) & KEY_MASK) >= T0) << (4 * j + 3);
                 rv[j] = a;
             }
-            stream_tile_record(p, w, flags);
-            if (hist && flags) {
-#pragma unroll
-                for (int j = 0; j < WT_VECS; ++j) {
-                    if ((flags >> (4 * j)) & 0xFu) {
-                        if ((flags >> (4 * j)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].x, T0, sh)], 1u);
-                        if ((flags >> (4 * j + 1)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].y, T0, sh)], 1u);
-                        if ((flags >> (4 * j + 2)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].z, T0, sh)], 1u);
-                        if ((flags >> (4 * j + 3)) & 1u) atomicAdd(&S.r1[stream_rel_bin(rv[j].w, T0, sh)], 1u);
-                    }
-                }
-            }
+            stream_tile_record<true>(p, w, flags, rv, hist, S.r1, T0, sh);
         } else {
-            stream_tile_record(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi, sh));
+            stream_tile_record<false>(p, w, stream_tile_general<VEC>(p, S, base, l_lo, l_hi, sh),
+                                      nullptr);
         }
         w = stat_next ? w + GW : R * GW + __shfl_sync(0xFFFFFFFFu, ticket, 0);
     }
-    if (hist) {
-        __syncthreads();
+    __syncthreads();
+    if (hist)
         for (int i = tid; i < REL_BINS; i += blockDim.x)
             if (S.r1[i]) atomicAdd(&p.r1[i], S.r1[i]);
-    }
+    if (tid == 0) span_last(p.ctrl, SPAN_STREAM_LAST);
 }
 
 }  // namespace tke

@@ -1084,7 +1084,19 @@ int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns) {
     for (int i = 0; i < 8; ++i)
         ns[i] = c.t_phase[i] ? (int64_t)(c.t_phase[i] - c.t_phase[0]) : -1;
     for (int i = 0; i < 3; ++i) ns[8 + i] = m0.t_ns[2] ? (int64_t)m0.t_ns[i] : -1;
-    ns[11] = -1;
+    // spans over all blocks, from the first streaming block past its wait
+    const uint64_t s0 = c.t_span[SPAN_STREAM_FIRST] ? ~c.t_span[SPAN_STREAM_FIRST] : 0;
+    const uint64_t sel0 = c.t_span[SPAN_SELECT_FIRST] ? ~c.t_span[SPAN_SELECT_FIRST] : 0;
+    auto rel = [&](uint64_t t) { return (s0 && t) ? (int64_t)(t - s0) : (int64_t)-1; };
+    ns[11] = rel(c.t_span[SPAN_STREAM_LAST]);
+    ns[12] = rel(sel0);
+    ns[13] = rel(c.t_phase[0]);
+    ns[14] = rel(c.t_span[SPAN_SELECT_LAST]);
+    ns[15] = rel(c.t_span[SPAN_START_LAST]);
+    ns[16] = rel(c.t_span[SPAN_OFFSET_LAST]);
+    ns[17] = rel(c.t_span[SPAN_GATHER_LAST]);
+    ns[18] = rel(c.t_span[SPAN_BAR2_LAST]);
+    ns[19] = -1;
     return TOPK_EF_OK;
 }
 

@@ -295,7 +295,7 @@ int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
 
 /*
  * Diagnostics of the last compress call on `ws` (synchronises `stream`), in
- * nanoseconds; -1 for a step that did not run.  `ns` is host memory of 12
+ * nanoseconds; -1 for a step that did not run.  `ns` is host memory of 20
  * int64.  ns[0..7]: block 0 of the select kernel, from the kernel's start:
  *   candidate path: ns[4] offset look-back done, ns[5] gather done,
  *     ns[1] first grid barrier, ns[2] second grid barrier, ns[3] barrier of
@@ -304,7 +304,14 @@ int topk_ef_path_info(const void* ws, void* stream, int64_t* info);
  *   rescan fallback: ns[1] gather barrier, ns[3..5] the barriers after
  *     digit passes 1..3, ns[6] the count barrier, ns[7] end.
  * ns[8..10]: the sampling block of the first tensor, from its start: samples
- * loaded, first histogram level resolved, end.  ns[11] is reserved (-1).
+ * loaded, first histogram level resolved, end.
+ * ns[11..14], over all blocks and from the moment the first block of the
+ * streaming pass got past its wait on the setup kernel: the last streaming
+ * block done, the first select (or threshold) block started, block 0 of that
+ * kernel started, its last block done; then, latest over the blocks of that
+ * kernel: block started, output offset known (candidate path), candidates
+ * gathered, arrived at the barrier after the entry lists.  ns[19] is
+ * reserved (-1).
  */
 int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns);
 

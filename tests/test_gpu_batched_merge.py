@@ -51,6 +51,36 @@ def test_batched_vgg16_scaled_down():
     run_batched_steps(grads, offsets, ks, LR, ws=_wsb(offsets, ks))
 
 
+def test_batched_dense_tiles():
+    """Tiles of the streaming pass with far more than 32 candidates, which
+    the select rescans: four small tensors of equal magnitudes (random
+    signs, a few doubled), sharing tiles, where every element is a
+    candidate and the ties at the k-th magnitude go to the lower indices;
+    and a large tensor whose 25,000 largest entries sit in one contiguous
+    block.  The candidate path must hold (no rescan of the residual)."""
+    rng = np.random.default_rng(21)
+    sizes = [700, 1500, 3000, 5001, 130_000, 9]
+    ks = [50, 1500, 100, 2600, 20_000, 0]
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    grads = []
+    for s in range(2):
+        g = np.empty(int(offsets[-1]), np.float32)
+        for l in range(4):
+            a, b = int(offsets[l]), int(offsets[l + 1])
+            m = np.where(rng.random(b - a) < 0.5, -1.0, 1.0).astype(np.float32)
+            m[rng.choice(b - a, max(1, (b - a) // 100), replace=False)] *= np.float32(2.0)
+            g[a:b] = m
+        a, b = int(offsets[4]), int(offsets[5])
+        g[a:b] = rng.laplace(0, 1e-3, b - a).astype(np.float32)
+        g[a + 40_000:a + 65_000] = (rng.uniform(0.5, 1.5, 25_000) *
+                                    np.where(rng.random(25_000) < 0.5, -1, 1)).astype(np.float32)
+        g[offsets[5]:] = rng.laplace(0, 1.0, sizes[5]).astype(np.float32)
+        grads.append(g)
+    ws = _wsb(offsets, ks)
+    run_batched_steps(grads, offsets, ks, LR, ws=ws)
+    assert ef.topk_ef_path_info(ws)["fallback"] == 0
+
+
 def test_batched_many_tensors():
     """More tensors than one launch group holds (600 > 256)."""
     rng = np.random.default_rng(9)
