@@ -43,6 +43,13 @@ constexpr int EMIT_TILE = SEL_THREADS * EMIT_PER_THREAD;
 constexpr uint32_t ENT_PER = 4096;
 // Tiles of more than WT_THREAD candidates a warp gathers at once.
 constexpr int OVF_U = 4;
+// Rescan queue of the hard-threshold step: 16-byte entries (tile + 1, 0,
+// output position) in the per-tensor histogram words, which that step does
+// not use.
+constexpr uint32_t RQ_CAP = (uint32_t)CHIST_WORDS / 4;
+// Its counters (slots reserved, slots handed out, blocks done queueing) in
+// words of the control block that only merge calls use otherwise.
+constexpr int RQ_RESERVE = 0, RQ_HEAD = 1, RQ_DONE = 2;
 
 struct Slot {
     int32_t l_first, l_last;
@@ -189,6 +196,7 @@ struct CompressSrc {
     uint32_t* ent_cnt;           // [T] their lengths
     uint64_t* agg;               // [grid] each block's candidate count + 1 (0: not yet)
     int32_t r1_done;             // one tensor: the streaming pass built relative digit 1
+    uint4* rq;                   // hard threshold: rescan queue [RQ_CAP] (null: none)
     int32_t force_dense;
     int32_t dense;               // decided inside the kernel
 
@@ -712,6 +720,66 @@ __device__ __noinline__ void gather_rescan(const RescanArgs src, SelShared& S, u
     }
 }
 
+// Hard threshold: queue tile w (output position pos) for rescanning by any
+// warp (one warp, lane 0 writes).  False if the queue is full.
+__device__ __forceinline__ bool rq_push(const CompressSrc& src, const SelCommon& cm, uint32_t w,
+                                        uint64_t pos) {
+    uint32_t slot = 0;
+    if (lane_id() == 0) slot = atomicAdd(&cm.ctrl->merge_bar[RQ_RESERVE], 1u);
+    slot = __shfl_sync(0xFFFFFFFFu, slot, 0);
+    if (slot >= RQ_CAP) return false;
+    if (lane_id() == 0) {
+        uint32_t* e = reinterpret_cast<uint32_t*>(src.rq + slot);
+        e[2] = (uint32_t)pos;
+        e[3] = (uint32_t)(pos >> 32);
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(e), "r"(w + 1u) : "memory");
+    }
+    return true;
+}
+
+// Hard threshold: the warp takes queued tiles and rescans them while the
+// queue holds untaken ones.  A ticket (atomic add) is taken only when one
+// looked free; a ticket whose slot is not reserved yet is kept until its
+// slot is filled or every block has finished queueing, so none is lost.  The
+// block that queued a tile takes from the queue afterwards itself.
+__device__ void rq_drain(const CompressSrc& src, const SelCommon& cm, SelShared& S) {
+    uint32_t* head = &cm.ctrl->merge_bar[RQ_HEAD];
+    const volatile uint32_t* resv = &cm.ctrl->merge_bar[RQ_RESERVE];
+    const uint32_t* done = &cm.ctrl->merge_bar[RQ_DONE];
+    for (;;) {
+        uint32_t w1 = 0, plo = 0, phi = 0;
+        if (lane_id() == 0) {
+            const uint32_t r = min(*resv, RQ_CAP);
+            const uint32_t h = *reinterpret_cast<volatile uint32_t*>(head);
+            if (h < r) {
+                const uint32_t t = atomicAdd(head, 1u);
+                if (t < RQ_CAP) {
+                    const uint32_t* e = reinterpret_cast<const uint32_t*>(src.rq + t);
+                    uint32_t it = 0;
+                    for (;;) {
+                        if ((w1 = ld_acquire_u32(e)) != 0) break;
+                        if (ld_acquire_u32(done) == gridDim.x && t >= *resv) break;
+                        if (++it > SPIN_LIMIT) {
+                            atomicOr(&cm.ctrl->status, ST_TIMEOUT);
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                    if (w1) {
+                        plo = e[2];
+                        phi = e[3];
+                    }
+                }
+            }
+        }
+        w1 = __shfl_sync(0xFFFFFFFFu, w1, 0);
+        if (w1 == 0) return;
+        const uint64_t pos = ((uint64_t)__shfl_sync(0xFFFFFFFFu, phi, 0) << 32) |
+                             __shfl_sync(0xFFFFFFFFu, plo, 0);
+        gather_rescan<true>(RescanArgs(src), S, w1 - 1u, pos, nullptr, 0);
+    }
+}
+
 // Candidates of warp tile w below element bound (one thread).
 __device__ uint32_t tile_count_below(const CompressSrc& src, const SelShared& S, uint32_t w,
                                      uint32_t cnt, int64_t bound) {
@@ -879,12 +947,23 @@ __device__ void gather_phase(CompressSrc& src, const SelCommon& cm, SelShared& S
                     store_warp_staged<kThr>(src, S, wo[u], S.ovf_pos[i], cn[u], o[u], v[u], s_r1, lc);
             }
         }
-        // more than WT_CAP: rescanned
-        for (uint32_t i = warp; i < novf; i += nwarps)
-            if (s_ovf_w[SEL_THREADS + i] > (uint32_t)WT_CAP)
-                gather_rescan<kThr>(RescanArgs(src), S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
+        // more than WT_CAP: rescanned (hard threshold: queued for any warp of
+        // the grid while the queue has room; dense tiles crowd into few blocks)
+        for (uint32_t i = warp; i < novf; i += nwarps) {
+            if (s_ovf_w[SEL_THREADS + i] <= (uint32_t)WT_CAP) continue;
+            if (kThr && src.rq && rq_push(src, cm, s_ovf_w[i], S.ovf_pos[i])) continue;
+            gather_rescan<kThr>(RescanArgs(src), S, s_ovf_w[i], S.ovf_pos[i], s_r1, lc);
+        }
         __syncthreads();
         run += piece;
+    }
+    if (kThr && src.rq) {
+        // this block has queued all its dense tiles
+        __syncthreads();
+        if (tid == 0)
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&cm.ctrl->merge_bar[RQ_DONE])
+                         : "memory");
+        rq_drain(src, cm, S);
     }
     my0 = before;
     my1 = before + mine;

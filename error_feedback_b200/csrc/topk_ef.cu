@@ -450,6 +450,7 @@ int threshold_call(const float* grad, float* resid, int64_t n, float lr, uint32_
     src.cand_idx = reinterpret_cast<uint32_t*>(out_idx);
     src.cand_val = out_val;
     src.cap = (uint64_t)std::min<int64_t>(max_out, n);
+    src.rq = reinterpret_cast<uint4*>(ws + L.hist);   // cleared by the setup kernel
     SelCommon cm;
     cm.ctrl = sp.ctrl;
     cm.bar = &sp.ctrl->bar;

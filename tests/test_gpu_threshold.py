@@ -66,6 +66,31 @@ def test_threshold_zero_all_pass():
     assert counts == [n, n]
 
 
+def test_dense_tiles_past_queue():
+    """More dense warp tiles than the rescan queue holds (3,906 > 3,072): the
+    overflow is rescanned by the blocks that found it."""
+    n = 4_000_000
+    rng = np.random.default_rng(5)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(2)]
+    counts = run_threshold_steps(grads, LR, 0.0, n)
+    assert counts == [n, n]
+
+
+def test_dense_block_region():
+    """Passing entries crowded into one contiguous region (as when the
+    entries past the cap keep growing): the region's tiles are rescanned by
+    warps all over the grid."""
+    n = 3_000_000
+    rng = np.random.default_rng(6)
+    grads = []
+    for _ in range(2):
+        g = (rng.standard_normal(n) * 0.01).astype(np.float32)
+        g[1_000_000:1_200_000] = rng.uniform(1.0, 2.0, 200_000).astype(np.float32)
+        grads.append(g)
+    counts = run_threshold_steps(grads, LR, 0.05, 150_000)
+    assert counts[0] >= 200_000
+
+
 def test_ties_at_threshold_and_specials():
     """Magnitudes exactly at the threshold pass; NaN, +-Inf and -0 follow the
     magnitude order; a negative threshold acts by magnitude."""
