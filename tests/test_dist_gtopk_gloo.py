@@ -113,3 +113,41 @@ def test_allreduce_matches_single_device_tournament(world):
         gi, gv = got[r]
         assert np.array_equal(gi, oi), r
         assert np.array_equal(gv.view(np.uint32), ov.view(np.uint32)), r
+
+
+def _single_rank_checks(port, q):
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    from error_feedback_b200.dist import gtopk_allreduce
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    errs = []
+    try:
+        i = torch.arange(4, dtype=torch.int32)
+        v = torch.ones(4, dtype=torch.float32)
+        for bad in [(i.long(), v, 4), (i, v.double(), 4), (i, v, 3), (i[:3], v, 3)]:
+            try:
+                gtopk_allreduce(*bad, n=10)
+                errs.append("accepted a bad argument")
+            except ValueError:
+                pass
+        # one rank: no exchange, the set comes back as a new tensor
+        gi, gv = gtopk_allreduce(i, v, 4, 10)
+        if not (torch.equal(gi, i) and torch.equal(gv, v)) or gi.data_ptr() == i.data_ptr():
+            errs.append("single rank result")
+    finally:
+        dist.destroy_process_group()
+    q.put(errs)
+
+
+def test_argument_checks_and_single_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_single_rank_checks, args=(_free_port(), q))
+    p.start()
+    errs = q.get(timeout=120)
+    p.join(60)
+    assert p.exitcode == 0 and errs == []
