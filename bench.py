@@ -752,6 +752,45 @@ def time_oracle(wl, steps, budget_elems):
     raise SystemExit("no oracle sample for this workload")
 
 
+def time_multithreaded(wl, budget_s=3.0):
+    """The OpenMP CPU baseline (cpu_baseline/, all host cores) on the same
+    workload: fused fmaf, per-thread bounded heaps, a merge of the heaps.
+    Returns None for workloads it does not cover."""
+    import cpu_baseline as mtb
+    nth = mtb.threads()
+    if isinstance(wl, FlatCompress):
+        ns = int(min(wl.n, 256 << 20))
+        ks = ns // max(1, round(wl.n / max(wl.k, 1))) if wl.k else 0
+        g = wl.make_grad(0)[:ns].copy()
+        res = np.zeros(ns, np.float32)
+        mtb.compress(g, res, LR, ks, nth)          # warm-up (page faults, threads)
+        steps, t0 = 0, time.perf_counter()
+        while True:
+            mtb.compress(g, res, LR, ks, nth)
+            steps += 1
+            dt = time.perf_counter() - t0
+            if dt > budget_s or steps >= 200:
+                break
+        sample = f"{steps} EF steps on the first {ns} elements (k={ks}), {nth} threads"
+        return steps * (12 * ns + 8 * ks) / dt, steps * ns / dt, nth, sample, dt
+    if isinstance(wl, BatchedCompress):
+        g, off, ks = datagen.vgg16_bucket(0)
+        res = np.zeros(g.size, np.float32)
+        steps, t0 = 0, time.perf_counter()
+        while True:
+            for l in range(len(ks)):
+                a, b = int(off[l]), int(off[l + 1])
+                r = res[a:b]
+                mtb.compress(g[a:b], r, LR, int(ks[l]), nth)
+            steps += 1
+            dt = time.perf_counter() - t0
+            if dt > budget_s:
+                break
+        return (steps * wl.bytes_per_step / dt, steps * wl.elems_per_step / dt, nth,
+                f"{steps} EF steps on the full bucket, {nth} threads", dt)
+    return None
+
+
 def cpu_baseline(wl, args):
     budget = wl.elems_per_step if isinstance(wl, FlatCompress) else None
     if isinstance(wl, FlatCompress):
@@ -761,9 +800,17 @@ def cpu_baseline(wl, args):
     else:
         steps = 1
         dt, sample, bps, eps = time_oracle(wl, steps, budget)
-    return {"value": round(steps * bps / dt / 1e9, 4), "unit": "GB/s",
-            "elems_per_s": round(steps * eps / dt, 1), "cores": 1, "kind": "oracle",
-            "sample": sample, "seconds": round(dt, 3)}
+    out = {"value": round(steps * bps / dt / 1e9, 4), "unit": "GB/s",
+           "elems_per_s": round(steps * eps / dt, 1), "cores": 1, "kind": "oracle",
+           "sample": sample, "seconds": round(dt, 3)}
+    mt = time_multithreaded(wl)
+    if mt is not None:
+        gbs, eps_mt, nth, sample_mt, dt_mt = mt
+        out["multithreaded"] = {"value": round(gbs / 1e9, 4), "unit": "GB/s",
+                                "elems_per_s": round(eps_mt, 1), "cores": nth,
+                                "kind": "openmp fmaf + per-thread heaps (cpu_baseline/)",
+                                "sample": sample_mt, "seconds": round(dt_mt, 3)}
+    return out
 
 
 def run_reference(args):
