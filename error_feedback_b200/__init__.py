@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.topk_ef_compress_static.argtypes = [_vp, _vp, _i64, ctypes.c_float, _i64, _vp, _vp,
                                               _vp]
         L.topk_ef_compress_static.restype = ctypes.c_int
+        L.topk_ef_static_last_device_status.argtypes = [_vp]
+        L.topk_ef_static_last_device_status.restype = ctypes.c_int
         L.topk_ef_threshold_workspace_bytes.argtypes = [_i64]
         L.topk_ef_threshold_workspace_bytes.restype = _sz
         L.topk_ef_threshold.argtypes = [_vp, _vp, _i64, ctypes.c_float, ctypes.c_float, _i64,
@@ -196,6 +198,12 @@ def topk_ef_compress_static(grad, residual, lr, k, out_idx=None, out_val=None, s
                                        out_idx.data_ptr(), out_val.data_ptr(), _stream(stream))
     _check(rc, "topk_ef_compress_static")
     return out_idx, out_val
+
+
+def topk_ef_static_last_device_status(stream=None) -> int:
+    """Device-side status of the last topk_ef_compress_static call on the
+    current device (synchronises the stream)."""
+    return int(lib().topk_ef_static_last_device_status(_stream(stream)))
 
 
 def topk_ef_threshold_workspace_bytes(n: int) -> int:

@@ -48,6 +48,8 @@ constexpr uint32_t ST_INCONSISTENT = 4u;    // a count did not add up
 
 // Bounded waits: iterations of ~64 ns sleeps before a wait gives up.
 constexpr uint32_t SPIN_LIMIT = 1u << 22;
+// ... and the time after which a grid barrier gives up, whichever comes first.
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 
 // Control block at the start of every workspace.
 struct Ctrl {
@@ -60,7 +62,8 @@ struct Ctrl {
     uint32_t kernels;       // kernels the call launched
     uint32_t r2_path;       // compress: a tensor's k-th bin was too full for its entry list
     uint32_t merge_bar[32]; // grid barrier counters, one per merge round
-    uint32_t pad1[6];
+    uint32_t stall;         // test hook: extra arrivals the flat select's barrier waits for
+    uint32_t pad1[5];
     uint64_t t_phase[8];    // select kernel: globaltimer at each phase (block 0)
     uint64_t t_span[8];     // globaltimer over all blocks (diagnostics): the first
                             // block of a kernel stores ~t (atomicMax of the
@@ -167,23 +170,28 @@ __device__ __forceinline__ T block_sum(T v, T* s) {
     return tot;
 }
 
-// Grid-wide barrier for a co-resident (cooperative) grid.  `counter` starts
-// at 0 for the launch and only grows; `epoch` counts the barriers this block
-// has passed.  Gives up after SPIN_LIMIT waits, records ST_TIMEOUT and
-// returns false: every block then leaves the kernel.
+// Grid-wide barrier for a co-resident grid.  `counter` starts at 0 for the
+// launch and only grows; `epoch` counts the barriers this block has passed.
+// Gives up after SPIN_LIMIT waits or WAIT_LIMIT_NS, whichever comes first,
+// records ST_TIMEOUT and returns false: every block then leaves the kernel.
+// `extra` arrivals beyond the grid are waited for in addition (0; a test
+// hook sets 1 so that the wait runs out).
 __device__ __forceinline__ bool grid_barrier(uint32_t* counter, uint32_t& epoch,
-                                             uint32_t* status, int* s_flag) {
+                                             uint32_t* status, int* s_flag, uint32_t extra = 0) {
     __syncthreads();
     if (threadIdx.x == 0) {
         epoch += 1;
-        const uint32_t target = epoch * gridDim.x;
+        const uint32_t target = epoch * gridDim.x + extra;
         // release: the block's writes (ordered before by the block barrier)
         // are visible to whoever acquires the count
         asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
         uint32_t it = 0;
         int ok = 1;
+        uint64_t t0 = 0;
         while (ld_acquire_u32(counter) < target) {
-            if (++it > SPIN_LIMIT) {
+            ++it;
+            if (it == 33) t0 = global_ns();
+            if (it > SPIN_LIMIT || (it > 33 && (it & 63u) == 0 && global_ns() - t0 > WAIT_LIMIT_NS)) {
                 atomicOr(status, ST_TIMEOUT);
                 ok = 0;
                 break;

@@ -47,6 +47,20 @@ struct SegMeta {
 };
 static_assert(sizeof(SegMeta) == 48, "SegMeta layout");
 
+// Prefilter threshold for the next call on the same flat tensor: written by
+// the select kernel of a call that took the candidate path, used by the next
+// call's setup kernel instead of sampling when the tag matches (same n, k,
+// lr and residual).  The result never depends on it: a threshold that turns
+// out too high or too low sends the call to the rescan of the residual, and
+// that call clears the hint.
+struct Hint {
+    uint64_t tag;       // 0: none
+    uint32_t T0;
+    uint32_t shift;
+    uint32_t pad[12];
+};
+static_assert(sizeof(Hint) == 64, "Hint layout");
+
 template <int TCAP>
 struct SetupParams {
     const float* grad;
@@ -69,6 +83,9 @@ struct SetupParams {
     uint16_t sampled[TCAP]; // i-th sampled tensor (block i samples it)
     int32_t has_fixed_T0;   // hard threshold: every tensor uses fixed_T0
     uint32_t fixed_T0;
+    const Hint* hint;       // one sampled tensor: the previous call's threshold
+    uint64_t hint_tag;      // ... used when its tag equals this (0: never)
+    uint32_t stall;         // test hook: Ctrl::stall
 };
 
 // Block i < n_sampled samples acc for the prefilter threshold T0 of the i-th
@@ -98,6 +115,23 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
         const int64_t n = p.off[l + 1] - off;
         const uint32_t m = p.m[l];
         const bool full = (int64_t)m == n;
+        if (p.hint != nullptr && p.hint_tag != 0) {
+            const Hint h = *p.hint;
+            if (h.tag == p.hint_tag) {
+                if (tid == 0) {
+                    SegMeta sm;
+                    memset(&sm, 0, sizeof(sm));
+                    sm.off = off;
+                    sm.n = n;
+                    sm.out_base = p.out_base[l];
+                    sm.k = p.k[l];
+                    sm.T0 = h.T0;
+                    sm.shift = h.shift;
+                    p.meta[l] = sm;
+                }
+                return;
+            }
+        }
         const uint64_t t_start = global_ns();
         for (int i2 = tid; i2 < SAMPLE_BINS; i2 += blockDim.x) hist[i2] = 0;
         // every element, or 128 runs of 64 consecutive elements; all loads
@@ -174,6 +208,7 @@ setup_kernel(const __grid_constant__ SetupParams<TCAP> p) {
             memset(&c, 0, sizeof(c));
             c.cap = p.cap;
             c.kernels = p.kernels;
+            c.stall = p.stall;
             *p.ctrl = c;
         }
         for (int l = tid; l < p.T; l += blockDim.x) {

@@ -1368,31 +1368,18 @@ __device__ void compress_candidates(const CompressSrc& src, const SelCommon& cm,
 
 // ---------------------------------------------------------------- kernel
 
+// Standard-digit selection over the positions of src (the merge rounds, and
+// the compress step's rescan of the residual): digit passes first_digit..3
+// with a grid barrier after each, per-block (gt, eq) counts of the final key,
+// one more barrier, and the ordered emission.  Every block of the grid calls
+// it with the same epoch.
 template <class Src>
-__global__ void __launch_bounds__(SEL_THREADS)
-select_kernel(Src src, SelCommon cm) {
-    __shared__ SelShared S;
+__device__ void std_select(Src& src, const SelCommon& cm, uint32_t& epoch, SelShared& S,
+                           int first_digit) {
     const int tid = threadIdx.x;
     const int c = blockIdx.x;
     const int G = gridDim.x;
-    uint32_t epoch = 0;
     uint32_t* status = &cm.ctrl->status;
-    mark_phase(cm.ctrl, 0);
-    const BlockSpan block_span(cm.ctrl);
-
-    int first_digit;
-    if constexpr (std::is_same<Src, CompressSrc>::value) {
-        uint64_t my0, my1;
-        if (!compress_gather(src, cm, epoch, S, my0, my1)) return;
-        if (!src.dense) {
-            compress_candidates(src, cm, epoch, S, my0, my1);
-            return;
-        }
-        first_digit = 1;
-    } else {
-        src.fold_bad_input(cm.ctrl);
-        first_digit = src.d1_done ? 2 : 1;
-    }
     const int T = src.nseg();
     __syncthreads();
     for (int l = tid; l <= T; l += blockDim.x) S.seg[l] = src.seg_bound(l);
@@ -1515,6 +1502,30 @@ select_kernel(Src src, SelCommon cm) {
         emit_range(src, l, a, b, fs.prefix, fs.rem, src.seg_k(l), pg, pe, S);
     }
     mark_phase(cm.ctrl, 7);
+}
+
+template <class Src>
+__global__ void __launch_bounds__(SEL_THREADS)
+select_kernel(Src src, SelCommon cm) {
+    __shared__ SelShared S;
+    uint32_t epoch = 0;
+    mark_phase(cm.ctrl, 0);
+    const BlockSpan block_span(cm.ctrl);
+
+    int first_digit;
+    if constexpr (std::is_same<Src, CompressSrc>::value) {
+        uint64_t my0, my1;
+        if (!compress_gather(src, cm, epoch, S, my0, my1)) return;
+        if (!src.dense) {
+            compress_candidates(src, cm, epoch, S, my0, my1);
+            return;
+        }
+        first_digit = 1;
+    } else {
+        src.fold_bad_input(cm.ctrl);
+        first_digit = src.d1_done ? 2 : 1;
+    }
+    std_select(src, cm, epoch, S, first_digit);
 }
 
 }  // namespace tke

@@ -182,6 +182,8 @@ stream_kernel(const __grid_constant__ StreamParams p) {
             }
         }
     }
+    // the select kernel may be scheduled now (it waits for this grid to end)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");   // setup_kernel's results
     if (tid == 0) span_first(p.ctrl, SPAN_STREAM_FIRST);
     const uint32_t lane = lane_id();

@@ -1,7 +1,9 @@
 // Host side of the C ABI declared in include/topk_ef.h: argument checks,
 // workspace layout and the launch sequence of each call.
 //
-//   topk_ef_compress / _batched:  setup_kernel -> stream_kernel -> select_kernel
+//   topk_ef_compress / _batched:  setup_kernel -> stream_kernel -> select kernel
+//                                 (flat_select_kernel for a single tensor,
+//                                 select_kernel<CompressSrc> for a bucket)
 //   gtopk_merge:                  merge_setup_kernel -> (merge_round_kernel ->
 //                                 select_kernel) per tournament round
 //
@@ -25,6 +27,7 @@
 #include "kernels_select.cuh"
 #include "kernels_sparse.cuh"
 #include "kernels_merge_cluster.cuh"
+#include "kernels_flat.cuh"
 
 using namespace tke;
 
@@ -90,6 +93,7 @@ struct DevFacts {
     int k1_blocks = 0;       // resident stream_kernel blocks per SM
     int selc_blocks = 0;     // resident select_kernel<CompressSrc> blocks per SM
     int selm_blocks = 0;     // resident select_kernel<MergeSrc> blocks per SM
+    int fs_blocks = 0;       // resident flat_select_kernel blocks per SM
 };
 
 std::mutex g_facts_mu;
@@ -114,6 +118,13 @@ int device_facts(DevFacts* out) {
             return cuda_fail(e);
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                  &f.selm_blocks, select_kernel<MergeSrc>, SEL_THREADS, 0)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaFuncSetAttribute(flat_select_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)sizeof(FlatShared))) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                 &f.fs_blocks, flat_select_kernel, FS_THREADS, sizeof(FlatShared))) != cudaSuccess)
             return cuda_fail(e);
         if (f.sms <= 0 || f.k1_blocks <= 0 || f.selc_blocks <= 0 || f.selm_blocks <= 0)
             return TOPK_EF_ERR_CUDA;
@@ -193,7 +204,7 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
 
 // Workspace layout of one compress group (<= TCAP_LARGE tensors).
 struct CLayout {
-    size_t ctrl, meta, zero_begin, cand_start, ent_cnt, agg, hist, zero_end, wt_count, wt_off,
+    size_t ctrl, meta, hint, zero_begin, cand_start, ent_cnt, agg, hist, zero_end, wt_count, wt_off,
         ent, slots, cand_idx, cand_val, total;
     int64_t cap;
     uint32_t num_wt;
@@ -211,6 +222,8 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + sizeof(Ctrl));
     L.meta = o;
     o = align_up(o + T * sizeof(SegMeta));
+    L.hint = o;
+    o = align_up(o + sizeof(Hint));
     L.zero_begin = o;
     L.cand_start = o;
     o = align_up(o + (T + 1) * sizeof(int64_t));
@@ -279,7 +292,8 @@ size_t groups_workspace(const std::vector<Group>& groups) {
 template <int TCAP>
 cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float* grad,
                          const float* resid, float lr, bool force_t0_zero, uint32_t kernels,
-                         cudaStream_t st, const uint32_t* fixed_T0 = nullptr) {
+                         cudaStream_t st, const uint32_t* fixed_T0 = nullptr,
+                         uint64_t hint_tag = 0, uint32_t stall = 0) {
     SetupParams<TCAP> p;
     memset(&p, 0, sizeof(p));
     if (fixed_T0) {
@@ -298,6 +312,12 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
     p.meta = reinterpret_cast<SegMeta*>(ws + L.meta);
     p.zero_ptr = reinterpret_cast<uint4*>(ws + L.zero_begin);
     p.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
+    p.stall = stall;
+    // a single tensor whose threshold comes from a true sample may take the
+    // previous call's instead
+    p.hint = reinterpret_cast<const Hint*>(ws + L.hint);
+    p.hint_tag = (g.plans.size() == 1 && g.plans[0].m == (uint32_t)SAMPLE_M && !force_t0_zero)
+                     ? hint_tag : 0;
     int ns = 0;
     for (int l = 0; l < T; ++l) {
         const TensorPlan& t = g.plans[l];
@@ -372,30 +392,58 @@ CompressSrc make_src(const Group& g, const CLayout& L, char* ws, const StreamPar
     return src;
 }
 
+// Tag of a flat compress call for the threshold hint: the next call may use
+// this call's threshold only for the same residual, n, k and lr.
+uint64_t hint_tag_of(const float* resid, int64_t n, uint32_t k, float lr) {
+    auto mix = [](uint64_t x) {
+        x += 0x9E3779B97F4A7C15ull;
+        x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+        x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+        return x ^ (x >> 31);
+    };
+    uint32_t lb;
+    memcpy(&lb, &lr, sizeof lb);
+    uint64_t h = mix((uint64_t)(uintptr_t)resid);
+    h = mix(h ^ (uint64_t)n);
+    h = mix(h ^ ((uint64_t)k << 32 | lb));
+    return h ? h : 1;
+}
+
 int compress_group(const Group& g, const float* grad, float* resid, float lr, int32_t* out_idx,
                    float* out_val, char* ws, cudaStream_t st, const DevFacts& f, int flags) {
     const CLayout L = compress_layout(g.N, g.plans);
     const int T = (int)g.plans.size();
     const bool force_dense = (flags & 1) != 0;
     const bool force_t0 = (flags & 2) != 0;
-    const uint32_t kernels = g.N > 0 ? 3u : 1u;
+    const uint32_t stall = (flags & 4) != 0 ? 1u : 0u;
     const float* gg = grad + g.base;
     float* rg = resid + g.base;
+    // A single tensor takes flat_select_kernel, one block per SM, when its
+    // candidate capacity is within what that grid stages in one round per
+    // block; a bucket (or a huge tensor) takes the segmented select.
+    const int G_flat = std::min(SLOT_MAX, f.sms);
+    const bool flat = T == 1 && f.fs_blocks >= 1 && L.cap <= (int64_t)G_flat * FS_CAND;
+    const bool flat_skip = flat && g.plans[0].k == 0;   // nothing to select
+    const uint32_t kernels = g.N > 0 ? (flat_skip ? 2u : 3u) : 1u;
+    const uint64_t tag = flat && !force_t0 && !force_dense
+                             ? hint_tag_of(rg, g.N, g.plans[0].k, lr) : 0;
     trace_before(st, "setup_kernel");
     cudaError_t e = T <= TCAP_SMALL
-                        ? launch_setup<TCAP_SMALL>(g, L, ws, gg, rg, lr, force_t0, kernels, st)
+                        ? launch_setup<TCAP_SMALL>(g, L, ws, gg, rg, lr, force_t0, kernels, st,
+                                                   nullptr, tag, stall)
                         : launch_setup<TCAP_LARGE>(g, L, ws, gg, rg, lr, force_t0, kernels, st);
     trace_after(st);
     if (e != cudaSuccess) return cuda_fail(e);
     if (g.N == 0) return TOPK_EF_OK;
 
-    // a single tensor with a short candidate list: the streaming pass builds
-    // relative digit 1 and the select kernel saves a grid barrier; long
-    // lists would pay more in the streaming pass than the barrier costs
-    const bool build_r1 = T == 1 && L.cap <= ((int64_t)1 << 19);
+    // a single tensor: the streaming pass builds relative digit 1 (for the
+    // segmented select only when the candidate list is short; long lists
+    // would pay more in the streaming pass than the barrier it saves costs)
+    const bool build_r1 = T == 1 && (flat || L.cap <= ((int64_t)1 << 19));
     StreamParams sp;
     if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp, build_r1)) != cudaSuccess)
         return cuda_fail(e);
+    if (flat_skip) return TOPK_EF_OK;
     Ctrl* ctrl = sp.ctrl;
 
     CompressSrc src = make_src(g, L, ws, sp, rg);
@@ -408,6 +456,34 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     cm.ctrl = ctrl;
     cm.bar = &ctrl->bar;
     cm.slots = reinterpret_cast<Slot*>(ws + L.slots);
+    if (flat) {
+        // a normal launch chained to the streaming pass; its blocks exchange
+        // counts once through global memory, which needs the whole grid (one
+        // block per SM) resident: every wait in it is bounded
+        FlatParams fp;
+        fp.src = src;
+        // no dense list here: the bound on the candidates is what the grid
+        // stages in one round per block
+        fp.src.cap = (uint64_t)G_flat * FS_CAND;
+        fp.cm = cm;
+        fp.hint = reinterpret_cast<Hint*>(ws + L.hint);
+        fp.hint_tag = tag;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G_flat);
+        cfg.blockDim = dim3(FS_THREADS);
+        cfg.dynamicSmemBytes = sizeof(FlatShared);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        trace_before(st, "flat_select_kernel");
+        e = cudaLaunchKernelEx(&cfg, flat_select_kernel, fp);
+        trace_after(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        return TOPK_EF_OK;
+    }
     // one block per SM: cheaper grid barriers, no less bandwidth for the
     // small candidate list (the rescan fallback is still memory bound)
     const int G = std::min(SLOT_MAX, f.sms * std::min(1, f.selc_blocks));
@@ -718,6 +794,13 @@ int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float
     if (rc != TOPK_EF_OK) return rc;
     return topk_ef_compress(grad, residual, n, lr, k, out_idx, out_val, ws, STATIC_SCRATCH_BYTES,
                             stream);
+}
+
+int topk_ef_static_last_device_status(void* stream) {
+    void* ws = nullptr;
+    const int rc = static_scratch_addr(&ws);
+    if (rc != TOPK_EF_OK) return rc;
+    return topk_ef_last_device_status(ws, stream);
 }
 
 size_t topk_ef_threshold_workspace_bytes(int64_t n) {

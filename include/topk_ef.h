@@ -123,6 +123,19 @@ int topk_ef_compress_static(const float* grad, float* residual, int64_t n, float
                             int64_t k, int32_t* out_idx, float* out_val,
                             void* stream);
 
+/*
+ * Device-side status of the last topk_ef_compress_static call on the current
+ * device, the counterpart of topk_ef_last_device_status(ws, stream) for the
+ * library's scratch array (which the caller has no address of): synchronises
+ * `stream` and returns TOPK_EF_OK, TOPK_EF_ERR_DEVICE_TIMEOUT or
+ * TOPK_EF_ERR_INTERNAL (TOPK_EF_ERR_CUDA if the read-back failed).  Check it
+ * before using the outputs of a call that may have hit a bounded wait.  The
+ * device address of the array is looked up once per device and kept; after
+ * cudaDeviceReset it is stale (as is every other device pointer of the
+ * process), and neither call may be used again.
+ */
+int topk_ef_static_last_device_status(void* stream);
+
 /* ------------------------------------------------------- hard threshold */
 
 /* Workspace bytes for topk_ef_threshold on n elements; 0 for invalid n. */
@@ -319,8 +332,15 @@ int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns);
  * Test hook, process wide: bit 0 forces the full rescan fallback of the
  * compress calls; bit 1 forces the prefilter threshold of every tensor to 0
  * (every element a candidate, which overflows the candidate capacity for
- * large tensors and so also ends in the fallback).  0 restores normal
- * behaviour.  Returns the previous flags.
+ * large tensors and so also ends in the fallback); bit 2 makes the grid-wide
+ * exchange of a single-tensor compress call wait for one block more than
+ * the grid has, so that its bounded wait runs out (after about a second) and
+ * the call records TOPK_EF_ERR_DEVICE_TIMEOUT, with undefined outputs.  0
+ * restores normal behaviour.  Returns the previous flags.  The flags are
+ * process-wide state read by every call in the process (the library's only
+ * state outside the caller's workspace besides the tracing record and the
+ * scratch array of topk_ef_compress_static): set them only in tests, with no
+ * other calls in flight.
  */
 int topk_ef_set_test_flags(int flags);
 

@@ -59,11 +59,14 @@ def assert_same_step(step, gi, gv, gres, oi, ov, ores):
                              f"gpu {gres[bad[0]]!r} oracle {ores[bad[0]]!r}")
 
 
-def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=None):
+def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=None, n=None):
     """EF steps on the GPU and in the oracle; every step compared.
-    grads: list of float32 arrays (one per step).  Returns the GPU residual."""
+    grads: float32 arrays, one per step (a list, or any iterable when n is
+    given, so that full-size sequences need not be held at once).  Returns
+    the GPU residual."""
     o = oracle.get()
-    n = grads[0].size
+    if n is None:
+        n = grads[0].size
     ores = np.zeros(n, np.float32) if res0 is None else res0.copy()
     dres = to_dev(ores, offset_elems)
     for s, g in enumerate(grads):
@@ -77,6 +80,8 @@ def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=No
 
 
 def run_batched_steps(grads, offsets, ks, lr, res0=None, backend=0, ws=None):
+    """Batched EF steps on the GPU and in the oracle; every step compared.
+    grads: any iterable of float32 bucket arrays, one per step."""
     o = oracle.get()
     N = int(offsets[-1])
     ores = np.zeros(N, np.float32) if res0 is None else res0.copy()

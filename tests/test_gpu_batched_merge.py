@@ -94,13 +94,12 @@ def test_batched_many_tensors():
 
 def test_batched_vgg16_full():
     """The full VGG-16 bucket (16 tensors, 138,344,128 elements), per-tensor
-    k = ceil(n_l / 1000); the first 2 of the 5 EF steps."""
-    grads = []
-    for s in range(2):
-        g, offsets, ks = datagen.vgg16_bucket(s)
-        grads.append(g)
+    k = ceil(n_l / 1000); all 5 EF steps of the workload, every one compared
+    bit for bit."""
+    _, offsets, ks = datagen.vgg16_bucket(0)
     ws = _wsb(offsets, ks)
-    run_batched_steps(grads, offsets, ks, LR, backend=1, ws=ws)
+    run_batched_steps((datagen.vgg16_bucket(s)[0] for s in range(5)), offsets, ks, LR,
+                      backend=1, ws=ws)
     assert ef.topk_ef_path_info(ws)["fallback"] == 0
 
 

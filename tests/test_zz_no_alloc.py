@@ -48,6 +48,8 @@ def test_static_scratch_matches_workspace_call(n, k):
         vb = torch.empty(k, dtype=torch.float32, device="cuda")
         rc = _static_call(dg, res_st, k, ib, vb)
         assert rc == 0, ef.status_string(rc)
+        st = ef.lib().topk_ef_static_last_device_status(torch.cuda.current_stream().cuda_stream)
+        assert st == 0, ef.status_string(st)
         torch.cuda.synchronize()
         assert torch.equal(ia, ib), f"step {step}: indices differ"
         assert same_bits(va.cpu().numpy(), vb.cpu().numpy()).all(), f"step {step}: values differ"
