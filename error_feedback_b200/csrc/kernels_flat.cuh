@@ -376,6 +376,7 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
     __syncthreads();
     // the k-th key's bin b1, and the 2k-th key's bin for the next call's hint
     fs_find2(F.hist, k, 2 * k, F);
+    mark_phase(ctrl, 1);
     const FindResult f1 = F.fr1;
     const uint32_t total = F.total;
     const bool cand_ok = !src.force_dense && k > 0 && f1.ok && f1.bin != (uint32_t)(REL_BINS - 1) &&
@@ -413,8 +414,8 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
     for (uint32_t wr = w0; wr < w1;) {
         if (wr != w0) fs_load_chunk(src, wr + tid, w1, r);
         const uint32_t nt = fs_stage_round(src, F, wr, w1, r, T0, status);
+        if (rounds == 0) mark_phase(ctrl, 4);
         const uint32_t nc = F.nc;
-        uint32_t g = 0, in = 0;
         for (uint32_t p0 = 0; p0 < nc; p0 += FS_THREADS) {
             const uint32_t q = p0 + tid;
             bool hit = false;
@@ -422,7 +423,7 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
             if (q < nc) {
                 const uint32_t rel = key_of(F.cval[q]) - T0;
                 const uint32_t bin = min(rel >> sh, (uint32_t)(REL_BINS - 1));
-                g += bin > b1;
+                gt_b += bin > b1;
                 hit = bin == b1;
                 low = rel & lmask;
             }
@@ -434,19 +435,19 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
                 at = __shfl_sync(0xFFFFFFFFu, at, lead) + __popc(mk & ((1u << lane_id()) - 1u));
                 if (hit) {
                     if (at < ENT_PER) src.ent[at] = ((uint32_t)c << 12) | low;
-                    atomicAdd(src.h(0, CH_R2) + low, 1u);
-                    ++in;
+                    ++in_b;
                 }
             }
         }
-        gt_b += g;
-        in_b += in;
         ++rounds;
         nc_last = nc;
         wr += nt;
     }
-    gt_b = block_sum(gt_b, F.red);
-    in_b = block_sum(in_b, F.red);
+    {
+        const uint64_t both = block_sum(((uint64_t)gt_b << 32) | in_b, F.scan);
+        gt_b = (uint32_t)(both >> 32);
+        in_b = (uint32_t)both;
+    }
     if (tid == 0) {
         Slot sl;
         memset(&sl, 0, sizeof(sl));
@@ -454,21 +455,39 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         sl.eq_first = in_b;
         cm.slots[c] = sl;
     }
+    mark_phase(ctrl, 5);
     mark_last(ctrl, SPAN_GATHER_LAST);
     if (!grid_barrier(cm.bar, epoch, status, &S.flag, stall)) return;
     mark_phase(ctrl, 2);
 
-    // ---- B: T, the tie quota and this block's output offset
-    const uint32_t E = *reinterpret_cast<const volatile uint32_t*>(src.ent_cnt);
-    uint32_t Tk, q, before_gt, before_eq;
+    // ---- B: T, the tie quota and this block's output offset.  The entry
+    // words, their count and the earlier blocks' counts are loaded together
+    // (slots past the count hold stale words and are dropped).
     constexpr int EPT = (int)ENT_PER / FS_THREADS;
-    if (E <= ENT_PER) {
-        uint32_t ev[EPT];
+    uint32_t ev[EPT];
 #pragma unroll
-        for (int u = 0; u < EPT; ++u) {
-            const uint32_t i = (uint32_t)(tid + u * FS_THREADS);
-            ev[u] = i < E ? src.ent[i] : DEAD;
+    for (int u = 0; u < EPT; ++u) ev[u] = src.ent[tid + u * FS_THREADS];
+    const uint32_t E = *reinterpret_cast<const volatile uint32_t*>(src.ent_cnt);
+    uint32_t gt_slots = 0;
+    if (tid < 32) {
+        // warp 0: the counts above b1 of blocks [0, c), 8 loads per lane in flight
+        for (int j0 = 0; j0 < c; j0 += 256) {
+            uint32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + 32 * u + tid;
+                v[u] = j < c ? cm.slots[j].gt_first : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) gt_slots += v[u];
         }
+        gt_slots = warp_sum(gt_slots);
+    }
+    uint32_t Tk, q, before_gt, before_eq;
+    if (E <= ENT_PER) {
+#pragma unroll
+        for (int u = 0; u < EPT; ++u)
+            if ((uint32_t)(tid + u * FS_THREADS) >= E) ev[u] = DEAD;
         for (int i = tid; i < REL_BINS; i += FS_THREADS) F.hist[i] = 0;
         __syncthreads();
 #pragma unroll
@@ -483,7 +502,7 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         const uint32_t t = F.fr1.bin;
         Tk = T0 + (b1 << sh) + t;
         q = rem - F.fr1.above;
-        uint32_t g = 0, e = 0;
+        uint32_t g = tid == 0 ? gt_slots : 0u, e = 0;
 #pragma unroll
         for (int u = 0; u < EPT; ++u) {
             if (ev[u] != DEAD && (int)(ev[u] >> 12) < c) {
@@ -491,12 +510,37 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
                 e += (ev[u] & 4095u) == t;
             }
         }
-        before_gt = fs_slots_before(cm.slots, c, 2, F) + block_sum(g, F.red);
-        before_eq = block_sum(e, F.red);
+        const uint64_t both = block_sum(((uint64_t)g << 32) | e, F.scan);
+        before_gt = (uint32_t)(both >> 32);
+        before_eq = (uint32_t)both;
     } else {
-        // the k-th key's bin is crowded: global digit-2 histogram and exact
-        // counts of every block
+        // the k-th key's bin holds more candidates than the entry list: a
+        // global digit-2 histogram of the bin, then exact counts of every
+        // block (two more grid-wide steps)
         if (c == 0 && tid == 0) ctrl->r2_path = 1;
+        for (int i = tid; i < REL_BINS; i += FS_THREADS) F.hist[i] = 0;
+        __syncthreads();
+        for (uint32_t wr = w0, rr = 0; wr < w1; ++rr) {
+            uint32_t nt = 0, nc = nc_last;
+            if (rounds > 1) {
+                fs_load_chunk(src, wr + tid, w1, r);
+                nt = fs_stage_round(src, F, wr, w1, r, T0, status);
+                nc = F.nc;
+            }
+            for (uint32_t p0 = tid; p0 < nc; p0 += FS_THREADS) {
+                const uint32_t rel = key_of(F.cval[p0]) - T0;
+                if (min(rel >> sh, (uint32_t)(REL_BINS - 1)) == b1) atomicAdd(&F.hist[rel & lmask], 1u);
+            }
+            __syncthreads();
+            if (rounds == 1) break;
+            wr += nt;
+        }
+        {
+            uint32_t* g2 = src.h(0, CH_R2);
+            for (int i = tid; i < REL_BINS; i += FS_THREADS)
+                if (F.hist[i]) atomicAdd(&g2[i], F.hist[i]);
+        }
+        if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
         stage_words(F.hist, src.h(0, CH_R2), REL_BINS, REL_BINS);
         __syncthreads();
         fs_find2(F.hist, rem, rem, F);
@@ -518,12 +562,11 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
                 wr += nt;
             }
         }
-        g = block_sum(g, F.red);
-        e = block_sum(e, F.red);
+        const uint64_t both = block_sum(((uint64_t)g << 32) | e, F.scan);
         if (tid == 0) {
             Slot sl = cm.slots[c];
-            sl.gt_last = g;
-            sl.eq_last = e;
+            sl.gt_last = (uint32_t)(both >> 32);
+            sl.eq_last = (uint32_t)both;
             cm.slots[c] = sl;
         }
         if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
