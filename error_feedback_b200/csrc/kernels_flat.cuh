@@ -55,6 +55,7 @@ struct FlatShared {
     FindResult fr1, fr2;
     uint32_t total;
     uint32_t pre[2];
+    uint32_t crowd[4];                   // crowded path: T, tie quota, counts before the block
 };
 
 struct FlatParams {
@@ -337,6 +338,102 @@ __device__ __forceinline__ void fs_count_exact(const FlatShared& F, uint32_t nc,
     }
 }
 
+// The rescan of the residual when the candidates cannot hold the answer
+// (out of line: it is rare, and the main path's straight-line code is what
+// every block fetches).
+__device__ __noinline__ void fs_fallback(const FlatParams& p, SelShared& S) {
+    CompressSrc d = p.src;
+    const SelCommon cm = p.cm;
+    d.dense = 1;
+    uint32_t epoch = 0;
+    std_select(d, cm, epoch, S, 1);
+}
+
+// The k-th key's bin holds more candidates than the entry list (heavy ties
+// or a crowded bin): a global digit-2 histogram of the bin, then exact
+// counts of every block, two more grid-wide steps.  Out of line (rare).
+// out: T, the tie quota, this block's counts above / equal to T before it.
+// Returns false if a wait gave up or the counts did not add up.
+__device__ __noinline__ bool fs_crowded(const FlatParams& p, FlatShared& F, SelShared& S,
+                                        uint32_t epoch, uint32_t w0, uint32_t w1,
+                                        uint32_t rounds, uint32_t nc_last, uint32_t T0,
+                                        uint32_t sh, uint32_t b1, uint32_t rem) {
+    const CompressSrc& src = p.src;
+    const SelCommon& cm = p.cm;
+    const int tid = threadIdx.x, c = blockIdx.x;
+    uint32_t* status = &cm.ctrl->status;
+    const uint32_t lmask = (1u << sh) - 1u;
+    uint32_t Tk, q;
+    ChunkRegs r;
+    // the k-th key's bin holds more candidates than the entry list: a
+    // global digit-2 histogram of the bin, then exact counts of every
+    // block (two more grid-wide steps)
+    if (c == 0 && tid == 0) cm.ctrl->r2_path = 1;
+    for (int i = tid; i < REL_BINS; i += FS_THREADS) F.hist[i] = 0;
+    __syncthreads();
+    for (uint32_t wr = w0; wr < w1;) {
+        uint32_t nt = 0, nc = nc_last;
+        if (rounds > 1) {
+            fs_load_chunk(src, wr + tid, w1, r);
+            nt = fs_stage_round(src, F, wr, w1, r, T0, status);
+            nc = F.nc;
+        }
+        for (uint32_t p0 = tid; p0 < nc; p0 += FS_THREADS) {
+            const uint32_t rel = key_of(F.cval[p0]) - T0;
+            if (min(rel >> sh, (uint32_t)(REL_BINS - 1)) == b1) atomicAdd(&F.hist[rel & lmask], 1u);
+        }
+        __syncthreads();
+        if (rounds == 1) break;
+        wr += nt;
+    }
+    {
+        uint32_t* g2 = src.h(0, CH_R2);
+        for (int i = tid; i < REL_BINS; i += FS_THREADS)
+            if (F.hist[i]) atomicAdd(&g2[i], F.hist[i]);
+    }
+    if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return false;
+    stage_words(F.hist, src.h(0, CH_R2), REL_BINS, REL_BINS);
+    __syncthreads();
+    fs_find2(F.hist, rem, rem, F);
+    if (!F.fr1.ok) {
+        if (tid == 0) atomicOr(status, ST_INCONSISTENT);
+        return false;
+    }
+    Tk = T0 + (b1 << sh) + F.fr1.bin;
+    q = rem - F.fr1.above;
+    uint32_t g = 0, e = 0;
+    if (rounds == 1) {
+        fs_count_exact(F, nc_last, Tk, g, e);
+    } else {
+        for (uint32_t wr = w0; wr < w1;) {
+            fs_load_chunk(src, wr + tid, w1, r);
+            const uint32_t nt = fs_stage_round(src, F, wr, w1, r, T0, status);
+            fs_count_exact(F, F.nc, Tk, g, e);
+            __syncthreads();
+            wr += nt;
+        }
+    }
+    const uint64_t both = block_sum(((uint64_t)g << 32) | e, F.scan);
+    if (tid == 0) {
+        Slot sl = cm.slots[c];
+        sl.gt_last = (uint32_t)(both >> 32);
+        sl.eq_last = (uint32_t)both;
+        cm.slots[c] = sl;
+    }
+    if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return false;
+    mark_phase(cm.ctrl, 3);
+    const uint32_t bg = fs_slots_before(cm.slots, c, 4, F);
+    const uint32_t be = fs_slots_before(cm.slots, c, 5, F);
+    if (tid == 0) {
+        F.crowd[0] = Tk;
+        F.crowd[1] = q;
+        F.crowd[2] = bg;
+        F.crowd[3] = be;
+    }
+    __syncthreads();
+    return true;
+}
+
 __global__ void __launch_bounds__(FS_THREADS, 1)
 flat_select_kernel(const __grid_constant__ FlatParams p) {
     extern __shared__ __align__(16) unsigned char fs_smem[];
@@ -389,9 +486,7 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         // every block takes the same decision: the standard-digit rescan;
         // the threshold that led here is not offered to the next call
         if (c == 0 && tid == 0 && p.hint) p.hint->tag = 0;
-        CompressSrc d = src;
-        d.dense = 1;
-        std_select(d, cm, epoch, S, 1);
+        fs_fallback(p, S);
         return;
     }
     const uint32_t b1 = f1.bin;
@@ -514,65 +609,11 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         before_gt = (uint32_t)(both >> 32);
         before_eq = (uint32_t)both;
     } else {
-        // the k-th key's bin holds more candidates than the entry list: a
-        // global digit-2 histogram of the bin, then exact counts of every
-        // block (two more grid-wide steps)
-        if (c == 0 && tid == 0) ctrl->r2_path = 1;
-        for (int i = tid; i < REL_BINS; i += FS_THREADS) F.hist[i] = 0;
-        __syncthreads();
-        for (uint32_t wr = w0, rr = 0; wr < w1; ++rr) {
-            uint32_t nt = 0, nc = nc_last;
-            if (rounds > 1) {
-                fs_load_chunk(src, wr + tid, w1, r);
-                nt = fs_stage_round(src, F, wr, w1, r, T0, status);
-                nc = F.nc;
-            }
-            for (uint32_t p0 = tid; p0 < nc; p0 += FS_THREADS) {
-                const uint32_t rel = key_of(F.cval[p0]) - T0;
-                if (min(rel >> sh, (uint32_t)(REL_BINS - 1)) == b1) atomicAdd(&F.hist[rel & lmask], 1u);
-            }
-            __syncthreads();
-            if (rounds == 1) break;
-            wr += nt;
-        }
-        {
-            uint32_t* g2 = src.h(0, CH_R2);
-            for (int i = tid; i < REL_BINS; i += FS_THREADS)
-                if (F.hist[i]) atomicAdd(&g2[i], F.hist[i]);
-        }
-        if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
-        stage_words(F.hist, src.h(0, CH_R2), REL_BINS, REL_BINS);
-        __syncthreads();
-        fs_find2(F.hist, rem, rem, F);
-        if (!F.fr1.ok) {
-            if (tid == 0) atomicOr(status, ST_INCONSISTENT);
-            return;
-        }
-        Tk = T0 + (b1 << sh) + F.fr1.bin;
-        q = rem - F.fr1.above;
-        uint32_t g = 0, e = 0;
-        if (rounds == 1) {
-            fs_count_exact(F, nc_last, Tk, g, e);
-        } else {
-            for (uint32_t wr = w0; wr < w1;) {
-                fs_load_chunk(src, wr + tid, w1, r);
-                const uint32_t nt = fs_stage_round(src, F, wr, w1, r, T0, status);
-                fs_count_exact(F, F.nc, Tk, g, e);
-                __syncthreads();
-                wr += nt;
-            }
-        }
-        const uint64_t both = block_sum(((uint64_t)g << 32) | e, F.scan);
-        if (tid == 0) {
-            Slot sl = cm.slots[c];
-            sl.gt_last = (uint32_t)(both >> 32);
-            sl.eq_last = (uint32_t)both;
-            cm.slots[c] = sl;
-        }
-        if (!grid_barrier(cm.bar, epoch, status, &S.flag)) return;
-        mark_phase(ctrl, 3);
-        before_gt = fs_slots_before(cm.slots, c, 4, F);
-        before_eq = fs_slots_before(cm.slots, c, 5, F);
+        if (!fs_crowded(p, F, S, epoch, w0, w1, rounds, nc_last, T0, sh, b1, rem)) return;
+        Tk = F.crowd[0];
+        q = F.crowd[1];
+        before_gt = F.crowd[2];
+        before_eq = F.crowd[3];
     }
     mark_last(ctrl, SPAN_OFFSET_LAST);
     mark_phase(ctrl, 6);

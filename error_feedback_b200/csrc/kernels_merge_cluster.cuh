@@ -141,7 +141,9 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     const int tid = threadIdx.x;
     const int cr = (int)cl.block_rank();
     const int pair = blockIdx.x / CL;
-    // the previous round's sets and sizes (programmatic serialisation)
+    // the next round may be scheduled now; this one waits for the previous
+    // round's sets and sizes (programmatic serialisation)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const bool stamp = blockIdx.x == 0 && tid == 0;     // diagnostics: CTA 0's phases
     if (stamp) p.ctrl->t_phase[0] = global_ns();

@@ -1,10 +1,12 @@
 """gTopKAllReduce across the ranks of a torch.distributed process group.
 
-"A Distributed Synchronous SGD Algorithm with Global Top-k Sparsification"
-(Sections III-IV, gTopKAllReduce): after each worker has sparsified its
-gradient to k (index, value) pairs, the workers reduce their sets along a
-binary tree in log2 P rounds and the result, the global top-k set, is
-broadcast to all of them.
+"A Distributed Synchronous SGD Algorithm with Global Top-k Sparsification
+for Low Bandwidth Networks" (review page, method section 提出的方法: the
+global top-k is found by a tournament in O(log P) rounds, each worker
+exchanging one k-pair set per round; ABSTRACT: O(k log P) communication):
+after each worker has sparsified its gradient to k (index, value) pairs, the
+workers reduce their sets along a binary tree in log2 P rounds and the
+result, the global top-k set, is broadcast to all of them.
 
 Round r (step s = 2^r): rank i with i mod 2s == s sends its set to rank
 i - s and leaves the tree; rank i with i mod 2s == 0 and a partner i + s < P
@@ -14,10 +16,13 @@ lower index first, index-ascending).  These are the pairs and the round order
 of the single-device tournament (``gtopk_merge`` over P rows), so rank 0 ends
 with the same set, bit for bit.  Rank 0 then broadcasts it.
 
-Only the exchange happens here (torch.distributed send / recv / broadcast:
-NCCL for CUDA tensors, one k-pair set per message); every merge runs in the
-library's kernels.  ``merge`` may be replaced by a callable with the same
-contract, which the CPU tests use to check the exchange schedule with gloo.
+Only the exchange happens here (torch.distributed point-to-point and
+broadcast: NCCL for CUDA tensors, one k-pair set per message); every merge
+runs in the library's kernels.  A rank posts the receives of all its rounds
+before its first merge, so a partner's set travels while this rank is still
+merging earlier rounds: each round's transfer overlaps the merge before it.
+``merge`` may be replaced by a callable with the same contract, which the
+CPU tests use to check the exchange schedule with gloo.
 """
 import torch
 
@@ -76,15 +81,26 @@ def gtopk_allreduce(idx, val, k, n, group=None, merge=None, ws=None):
     if merge is None:
         merge = _device_merge(ws)
     cur_i, cur_v = idx.contiguous(), val.contiguous()
-    for kind, partner in tree_schedule(rank, world):
+    steps = tree_schedule(rank, world)
+    # every receive of this rank's tree, posted before the first merge
+    recvs = []
+    for kind, partner in steps:
+        if kind == "recv":
+            ri = torch.empty_like(cur_i)
+            rv = torch.empty_like(cur_v)
+            works = [dist.irecv(ri, src=glob(partner), group=group),
+                     dist.irecv(rv, src=glob(partner), group=group)]
+            recvs.append((ri, rv, works))
+    nr = 0
+    for kind, partner in steps:
         if kind == "send":
             dist.send(cur_i, dst=glob(partner), group=group)
             dist.send(cur_v, dst=glob(partner), group=group)
         else:
-            ri = torch.empty_like(cur_i)
-            rv = torch.empty_like(cur_v)
-            dist.recv(ri, src=glob(partner), group=group)
-            dist.recv(rv, src=glob(partner), group=group)
+            ri, rv, works = recvs[nr]
+            nr += 1
+            for w in works:
+                w.wait()
             cur_i, cur_v = merge(torch.stack([cur_i, ri]), torch.stack([cur_v, rv]), k, n)
     out_i = cur_i.clone() if rank == 0 else torch.empty_like(idx)
     out_v = cur_v.clone() if rank == 0 else torch.empty_like(val)

@@ -193,3 +193,45 @@ def test_bf16_ties_1p5b_full():
         assert same, f"step {step}: residuals differ"
     info = ef.topk_ef_path_info(ws)
     assert info["fallback"] == 0, info
+
+
+def test_index_width_boundary():
+    """n = 2^31 - 1, the largest n the int32 indices allow (indices up to
+    2^31 - 2; the last warp tile holds 1,023 elements).  The gradient, drawn
+    on the device, is small everywhere (|g| in [1e-4, 1e-2]) except the last
+    1,000 elements (|g| in [1, 2]), so the top k = 600 lie in that tail and the
+    oracle on the tail alone gives the expected output; the residual must be
+    RN(lr * g) = fmaf(lr, g, 0) everywhere except the 600 sent slots (+0),
+    checked in full on the device and on a 2^20-element sample against the
+    oracle's own accumulate.  One EF step from a zero residual."""
+    import oracle
+    n, k, tail = (1 << 31) - 1, 600, 1000
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2_147_483_647)
+    g = torch.empty(n, dtype=torch.float32, device="cuda")
+    g.uniform_(1e-4, 1e-2, generator=gen)
+    sign = torch.empty(n, dtype=torch.float32, device="cuda").bernoulli_(0.5, generator=gen)
+    g.mul_(sign.mul_(2).sub_(1))
+    del sign
+    rng = np.random.default_rng(31)
+    gt = (rng.uniform(1.0, 2.0, tail) * np.where(rng.random(tail) < 0.5, -1, 1)).astype(np.float32)
+    g[n - tail:] = torch.from_numpy(gt).cuda()
+    res = torch.zeros(n, dtype=torch.float32, device="cuda")
+    ws = _ws(n, k)
+    gi, gv = ef.topk_ef_compress(g, res, LR, k, ws=ws)
+    assert ef.topk_ef_last_device_status(ws) == 0
+    o = oracle.get()
+    rt = np.zeros(tail, np.float32)
+    oi, ov = o.compress(gt, rt, LR, k, 1)
+    assert np.array_equal(gi.cpu().numpy(), oi.astype(np.int64) + (n - tail))
+    assert np.array_equal(bits(gv.cpu().numpy()), bits(ov))
+    # the sample, against the oracle's accumulate (fmaf(lr, g, 0))
+    pos = torch.from_numpy(np.sort(rng.choice(n - tail, 1 << 20, replace=False))).cuda()
+    acc = o.accumulate(g[pos].cpu().numpy(), np.zeros(1 << 20, np.float32), LR)
+    assert np.array_equal(bits(res[pos].cpu().numpy()), bits(acc))
+    assert np.array_equal(bits(res[n - tail:].cpu().numpy()), bits(rt))
+    # everywhere: fmaf(lr, g, +0) = RN(lr * g) for these magnitudes (no
+    # product rounds to zero), +0 at the sent slots
+    want = g.mul_(LR)
+    want[gi.long()] = 0.0
+    assert torch.equal(want.view(torch.int32), res.view(torch.int32))
