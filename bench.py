@@ -553,6 +553,9 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     wl = make_workload(args.workload)
+    if args.no_flush and wl.flush:
+        wl.flush = False
+        wl.l2_kept = True
     wl.setup(rank, args.steps + args.warmup)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
@@ -680,6 +683,9 @@ def run_ours(args):
             "e2e": e2e,
             "clocks": clocks,
         }
+        if getattr(wl, "l2_kept", False):
+            line["config"]["l2"] = ("not flushed (--no-flush): the step's inputs stay in L2 and "
+                                    "the steps run back to back")
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(wl, args)
         print(json.dumps(line), flush=True)
@@ -863,6 +869,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="resnet50_mix")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-flush", action="store_true",
+                    help="do not flush L2 between steps of a workload smaller than L2 "
+                         "(steps then run back to back from L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-elems", type=int, default=0,
                     help="reference arm: elements per step (default: sized to ~1 min)")

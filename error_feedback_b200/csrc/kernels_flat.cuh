@@ -511,38 +511,34 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         const uint32_t nt = fs_stage_round(src, F, wr, w1, r, T0, status);
         if (rounds == 0) mark_phase(ctrl, 4);
         const uint32_t nc = F.nc;
-        for (uint32_t p0 = 0; p0 < nc; p0 += FS_THREADS) {
-            const uint32_t q = p0 + tid;
-            bool hit = false;
-            uint32_t low = 0;
-            if (q < nc) {
+        // count first, reserve this round's entries with one atomic, then
+        // list them (no dependent global atomic per pass)
+        uint32_t in_t = 0;
+        for (uint32_t q = tid; q < nc; q += FS_THREADS) {
+            const uint32_t bin = min((key_of(F.cval[q]) - T0) >> sh, (uint32_t)(REL_BINS - 1));
+            gt_b += bin > b1;
+            in_t += bin == b1;
+        }
+        uint32_t in_r;
+        uint32_t at = block_excl_scan(in_t, F.red, &in_r);
+        if (tid == 0) F.pre[1] = in_r ? atomicAdd(src.ent_cnt, in_r) : 0u;
+        __syncthreads();
+        at += F.pre[1];
+        if (in_t) {
+            for (uint32_t q = tid; q < nc; q += FS_THREADS) {
                 const uint32_t rel = key_of(F.cval[q]) - T0;
-                const uint32_t bin = min(rel >> sh, (uint32_t)(REL_BINS - 1));
-                gt_b += bin > b1;
-                hit = bin == b1;
-                low = rel & lmask;
-            }
-            const uint32_t mk = __ballot_sync(0xFFFFFFFFu, hit);
-            if (mk) {
-                const uint32_t lead = (uint32_t)(__ffs(mk) - 1);
-                uint32_t at = 0;
-                if (lane_id() == lead) at = atomicAdd(src.ent_cnt, (uint32_t)__popc(mk));
-                at = __shfl_sync(0xFFFFFFFFu, at, lead) + __popc(mk & ((1u << lane_id()) - 1u));
-                if (hit) {
-                    if (at < ENT_PER) src.ent[at] = ((uint32_t)c << 12) | low;
-                    ++in_b;
+                if (min(rel >> sh, (uint32_t)(REL_BINS - 1)) == b1) {
+                    if (at < ENT_PER) src.ent[at] = ((uint32_t)c << 12) | (rel & lmask);
+                    ++at;
                 }
             }
         }
+        in_b += in_r;
         ++rounds;
         nc_last = nc;
         wr += nt;
     }
-    {
-        const uint64_t both = block_sum(((uint64_t)gt_b << 32) | in_b, F.scan);
-        gt_b = (uint32_t)(both >> 32);
-        in_b = (uint32_t)both;
-    }
+    gt_b = block_sum(gt_b, F.red);
     if (tid == 0) {
         Slot sl;
         memset(&sl, 0, sizeof(sl));

@@ -3,7 +3,9 @@
 //
 //   topk_ef_compress / _batched:  setup_kernel -> stream_kernel -> select kernel
 //                                 (flat_select_kernel for a single tensor,
-//                                 select_kernel<CompressSrc> for a bucket)
+//                                 select_kernel<CompressSrc> for a bucket);
+//                                 a single small tensor: setup_kernel ->
+//                                 small_kernel
 //   gtopk_merge:                  merge_setup_kernel -> (merge_round_kernel ->
 //                                 select_kernel) per tournament round
 //
@@ -28,6 +30,7 @@
 #include "kernels_sparse.cuh"
 #include "kernels_merge_cluster.cuh"
 #include "kernels_flat.cuh"
+#include "kernels_small.cuh"
 
 using namespace tke;
 
@@ -94,6 +97,7 @@ struct DevFacts {
     int selc_blocks = 0;     // resident select_kernel<CompressSrc> blocks per SM
     int selm_blocks = 0;     // resident select_kernel<MergeSrc> blocks per SM
     int fs_blocks = 0;       // resident flat_select_kernel blocks per SM
+    int sk_blocks = 0;       // resident small_kernel blocks per SM
 };
 
 std::mutex g_facts_mu;
@@ -125,6 +129,12 @@ int device_facts(DevFacts* out) {
             return cuda_fail(e);
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                  &f.fs_blocks, flat_select_kernel, FS_THREADS, sizeof(FlatShared))) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaFuncSetAttribute(small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)sizeof(SmallShared))) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                 &f.sk_blocks, small_kernel, SK_THREADS, sizeof(SmallShared))) != cudaSuccess)
             return cuda_fail(e);
         if (f.sms <= 0 || f.k1_blocks <= 0 || f.selc_blocks <= 0 || f.selm_blocks <= 0)
             return TOPK_EF_ERR_CUDA;
@@ -422,6 +432,50 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     // candidate capacity is within what that grid stages in one round per
     // block; a bucket (or a huge tensor) takes the segmented select.
     const int G_flat = std::min(SLOT_MAX, f.sms);
+    // A single tensor that one wave of blocks holds in shared memory takes
+    // small_kernel (no prefilter, no separate select)
+    const int sm_cap = std::min(SLOT_MAX, f.sms);
+    const bool small = T == 1 && f.sk_blocks >= 1 && g.N > 0 && g.plans[0].k > 0 &&
+                       !force_dense && g.N <= (int64_t)sm_cap * SK_MAX;
+    if (small) {
+        trace_before(st, "setup_kernel");
+        cudaError_t e = launch_setup<TCAP_SMALL>(g, L, ws, grad + g.base, resid + g.base, lr,
+                                                 true, 2u, st, nullptr, 0, stall);
+        trace_after(st);
+        if (e != cudaSuccess) return cuda_fail(e);
+        const int G = (int)std::max<int64_t>(1, std::min<int64_t>(sm_cap,
+                                                   ceil_div64(g.N, SK_MIN_PER_BLOCK)));
+        SmallParams kp;
+        kp.grad = grad + g.base;
+        kp.resid = resid + g.base;
+        kp.n = g.N;
+        kp.lr = lr;
+        kp.k = g.plans[0].k;
+        kp.out_idx = out_idx + g.plans[0].out_base;
+        kp.out_val = out_val + g.plans[0].out_base;
+        kp.ctrl = reinterpret_cast<Ctrl*>(ws + L.ctrl);
+        static_assert(CH_R2 == CH_R1 + SK_BINS / 2 && CH_D1 == CH_R1 + SK_BINS &&
+                      CHIST_WORDS - CH_D1 >= 1024, "small-kernel histograms in the tensor's words");
+        kp.hist = reinterpret_cast<uint32_t*>(ws + L.hist) + CH_R1;
+        kp.hist2 = reinterpret_cast<uint32_t*>(ws + L.hist) + CH_D1;
+        kp.ent = reinterpret_cast<uint32_t*>(ws + L.ent);
+        kp.ent_cnt = reinterpret_cast<uint32_t*>(ws + L.ent_cnt);
+        kp.slots = reinterpret_cast<Slot*>(ws + L.slots);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G);
+        cfg.blockDim = dim3(SK_THREADS);
+        cfg.dynamicSmemBytes = sizeof(SmallShared);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        trace_before(st, "small_kernel");
+        e = cudaLaunchKernelEx(&cfg, small_kernel, kp);
+        trace_after(st);
+        return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
+    }
     const bool flat = T == 1 && f.fs_blocks >= 1 && L.cap <= (int64_t)G_flat * FS_CAND;
     const bool flat_skip = flat && g.plans[0].k == 0;   // nothing to select
     const uint32_t kernels = g.N > 0 ? (flat_skip ? 2u : 3u) : 1u;

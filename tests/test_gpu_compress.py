@@ -24,7 +24,9 @@ def test_flat_normal_1m():
     grads = [datagen.flat_normal(s) for s in range(3)]
     ws = _ws(n, k)
     run_compress_steps(grads, LR, k, ws=ws)
-    assert ef.topk_ef_path_info(ws)["fallback"] == 0
+    info = ef.topk_ef_path_info(ws)
+    # a tensor this small takes the one-kernel path (setup + small_kernel)
+    assert info["fallback"] == 0 and info["kernels"] == 2, info
 
 
 @pytest.mark.parametrize("n,k", [
@@ -47,7 +49,8 @@ def test_empty():
     assert i.numel() == 0 and ef.topk_ef_last_device_status(ws) == 0
 
 
-@pytest.mark.parametrize("n,k", [(200_001, 5000), (1_000_000, 123_457), (70_000, 1)])
+@pytest.mark.parametrize("n,k", [(200_001, 5000), (1_000_000, 123_457), (70_000, 1),
+                                 (3_000_001, 30_000), (2_600_000, 1)])
 def test_heavy_ties(n, k):
     """Magnitudes from a handful of values: the threshold is shared by
     thousands of entries and the lower indices must win."""
@@ -64,9 +67,10 @@ def test_all_equal_magnitude():
     run_compress_steps([g], np.float32(1.0), k, ws=_ws(n, k))
 
 
-def test_special_values():
-    """NaN, +-Inf, +-0 and subnormals mixed into a normal gradient."""
-    n, k = 120_001, 1200
+@pytest.mark.parametrize("n,k", [(120_001, 1200), (2_500_001, 2500)])
+def test_special_values(n, k):
+    """NaN, +-Inf, +-0 and subnormals mixed into a normal gradient (one size
+    for the one-kernel path, one for the streaming pass + select)."""
     rng = np.random.default_rng(5)
     g = rng.standard_normal(n).astype(np.float32)
     sp = np.array([np.nan, np.inf, -np.inf, 0.0, -0.0, 1e-45, -1e-45, 1e-40, 3e38, -3e38],
@@ -78,10 +82,10 @@ def test_special_values():
     run_compress_steps([g, g], np.float32(1.0), k, res0=res0, ws=_ws(n, k))
 
 
-@pytest.mark.parametrize("offset", [1, 2, 3])
-def test_unaligned_base(offset):
-    """grad/residual not 16-byte aligned: the scalar path must agree."""
-    n, k = 300_007, 301
+@pytest.mark.parametrize("offset,n,k", [(1, 300_007, 301), (2, 300_007, 301), (3, 300_007, 301),
+                                        (1, 2_600_003, 2600), (3, 2_600_003, 2600)])
+def test_unaligned_base(offset, n, k):
+    """grad/residual not 16-byte aligned: the scalar paths must agree."""
     rng = np.random.default_rng(offset)
     grads = [rng.standard_normal(n).astype(np.float32) for _ in range(2)]
     run_compress_steps(grads, LR, k, offset_elems=offset, ws=_ws(n, k))
