@@ -37,7 +37,9 @@ namespace tke {
 constexpr int FS_THREADS = 512;
 constexpr int FS_TILES = FS_THREADS;     // tiles per staging chunk, one per thread
 constexpr int FS_CAND = 12288;           // candidates staged per round
-constexpr int FS_BATCH = 4;              // candidate loads a thread keeps in flight
+constexpr int FS_WARPS = FS_THREADS / 32;
+constexpr int FS_BATCH = 8;              // tiles whose candidate loads a warp keeps in flight
+constexpr int FS_CBATCH = 4;             // candidate loads a thread keeps in flight
 constexpr int FS_EMIT = 4;               // staged positions per thread per emission step
 
 struct FlatShared {
@@ -48,6 +50,7 @@ struct FlatShared {
     uint32_t tstart[FS_TILES + 1];       // first staged position of each tile
     uint32_t tcnt[FS_TILES];
     uint16_t dense[FS_TILES];            // tiles of the round with more than WT_CAP candidates
+    uint32_t wbm[FS_WARPS * 32];         // per warp: bitmap of a tile's candidate offsets
     uint64_t scan[33];
     uint32_t red[33];
     uint32_t ndense, nt, nc;
@@ -227,41 +230,91 @@ __device__ uint32_t fs_stage_round(const CompressSrc& src, FlatShared& F, uint32
     }
     __syncthreads();
     const uint32_t nc = F.nc;
-    // sparse tiles: candidate-parallel; a thread keeps FS_BATCH value loads
-    // in flight
-    for (uint32_t p0 = tid; p0 < nc; p0 += FS_THREADS * FS_BATCH) {
-        uint32_t e[FS_BATCH], q[FS_BATCH];
-        float v[FS_BATCH];
+    if (nc <= 4 * nt) {
+        // sparse tiles, few candidates per tile on average: candidate-parallel (a
+        // thread finds its tile by binary search and ranks its offset among the
+        // tile's); a thread keeps FS_CBATCH value loads in flight
+        for (uint32_t p0 = tid; p0 < nc; p0 += FS_THREADS * FS_CBATCH) {
+            uint32_t e[FS_CBATCH], q[FS_CBATCH];
+            float v[FS_CBATCH];
 #pragma unroll
-        for (int u = 0; u < FS_BATCH; ++u) {
-            const uint32_t p = p0 + (uint32_t)u * FS_THREADS;
-            q[u] = 0xFFFFFFFFu;
-            e[u] = 0;
-            if (p < nc) {
-                // tile of position p: last t with tstart[t] <= p
-                uint32_t lo = 0, hi = nt;
-                while (hi - lo > 1) {
-                    const uint32_t mid = (lo + hi) >> 1;
-                    if (F.tstart[mid] <= p) lo = mid; else hi = mid;
+            for (int u = 0; u < FS_CBATCH; ++u) {
+                const uint32_t p = p0 + (uint32_t)u * FS_THREADS;
+                q[u] = 0xFFFFFFFFu;
+                e[u] = 0;
+                if (p < nc) {
+                    // tile of position p: last t with tstart[t] <= p
+                    uint32_t lo = 0, hi = nt;
+                    while (hi - lo > 1) {
+                        const uint32_t mid = (lo + hi) >> 1;
+                        if (F.tstart[mid] <= p) lo = mid; else hi = mid;
+                    }
+                    const uint32_t c = F.tcnt[lo];
+                    if (c <= (uint32_t)WT_CAP) {
+                        const uint16_t* ot = F.off + lo * WT_CAP;
+                        const uint32_t o = ot[p - F.tstart[lo]];
+                        uint32_t rank = 0;
+                        for (uint32_t j = 0; j < c; ++j) rank += ot[j] < o;
+                        q[u] = F.tstart[lo] + rank;
+                        e[u] = (wr + lo) * (uint32_t)WT + o;
+                    }
                 }
-                const uint32_t c = F.tcnt[lo];
-                if (c <= (uint32_t)WT_CAP) {
-                    const uint16_t* ot = F.off + lo * WT_CAP;
-                    const uint32_t o = ot[p - F.tstart[lo]];
-                    uint32_t rank = 0;
-                    for (uint32_t j = 0; j < c; ++j) rank += ot[j] < o;
-                    q[u] = F.tstart[lo] + rank;
-                    e[u] = (wr + lo) * (uint32_t)WT + o;
+            }
+#pragma unroll
+            for (int u = 0; u < FS_CBATCH; ++u) v[u] = q[u] != 0xFFFFFFFFu ? src.resid[e[u]] : 0.f;
+#pragma unroll
+            for (int u = 0; u < FS_CBATCH; ++u) {
+                if (q[u] != 0xFFFFFFFFu) {
+                    F.cidx[q[u]] = e[u];
+                    F.cval[q[u]] = v[u];
                 }
             }
         }
+    } else {
+        // sparse tiles, many candidates per tile on average: a warp per tile, lane i holding
+        // the tile's staged candidate i; its rank in index order comes from a
+        // bitmap of the tile's offsets (one bit per element, 32 words) and one
+        // warp scan of the words' popcounts.  A warp keeps the value loads of
+        // FS_BATCH tiles in flight.
+        {
+            const uint32_t lane = lane_id(), warp = warp_id();
+            uint32_t* bm = F.wbm + warp * 32;
+            for (uint32_t t0 = warp; t0 < nt; t0 += FS_WARPS * FS_BATCH) {
+                uint32_t o[FS_BATCH], cn[FS_BATCH];
+                float v[FS_BATCH];
 #pragma unroll
-        for (int u = 0; u < FS_BATCH; ++u) v[u] = q[u] != 0xFFFFFFFFu ? src.resid[e[u]] : 0.f;
+                for (int u = 0; u < FS_BATCH; ++u) {
+                    const uint32_t t = t0 + (uint32_t)u * FS_WARPS;
+                    cn[u] = t < nt ? F.tcnt[t] : 0u;
+                    if (cn[u] > (uint32_t)WT_CAP) cn[u] = 0;            // dense: rescanned below
+                    o[u] = lane < cn[u] ? (uint32_t)F.off[t * WT_CAP + lane] : 0xFFFFu;
+                }
 #pragma unroll
-        for (int u = 0; u < FS_BATCH; ++u) {
-            if (q[u] != 0xFFFFFFFFu) {
-                F.cidx[q[u]] = e[u];
-                F.cval[q[u]] = v[u];
+                for (int u = 0; u < FS_BATCH; ++u) {
+                    const uint32_t t = t0 + (uint32_t)u * FS_WARPS;
+                    v[u] = o[u] != 0xFFFFu ? src.resid[(size_t)(wr + t) * WT + o[u]] : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < FS_BATCH; ++u) {
+                    if (cn[u] == 0) continue;                           // warp-uniform
+                    const uint32_t t = t0 + (uint32_t)u * FS_WARPS;
+                    const bool mine = o[u] != 0xFFFFu;
+                    if (mine) atomicOr(&bm[o[u] >> 5], 1u << (o[u] & 31u));
+                    __syncwarp();
+                    const uint32_t w = bm[lane];
+                    bm[lane] = 0u;
+                    const uint32_t pc = (uint32_t)__popc(w);
+                    const uint32_t ex = warp_incl_scan(pc) - pc;
+                    const uint32_t wi = (o[u] >> 5) & 31u;
+                    const uint32_t wx = __shfl_sync(0xFFFFFFFFu, ex, wi);
+                    const uint32_t ww = __shfl_sync(0xFFFFFFFFu, w, wi);
+                    if (mine) {
+                        const uint32_t q = F.tstart[t] + wx + (uint32_t)__popc(ww & ((1u << (o[u] & 31u)) - 1u));
+                        F.cidx[q] = (wr + t) * (uint32_t)WT + o[u];
+                        F.cval[q] = v[u];
+                    }
+                    __syncwarp();
+                }
             }
         }
     }
@@ -470,6 +523,7 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
         s4[tid] = a;
         s4[tid + FS_THREADS] = b;
     }
+    for (int i = tid; i < FS_WARPS * 32; i += FS_THREADS) F.wbm[i] = 0u;
     __syncthreads();
     // the k-th key's bin b1, and the 2k-th key's bin for the next call's hint
     fs_find2(F.hist, k, 2 * k, F);
