@@ -60,6 +60,27 @@ def test_heavy_ties(n, k):
     run_compress_steps(grads, np.float32(1.0), k, ws=_ws(n, k))
 
 
+def test_concentrated_candidates():
+    """n = 3,000,017 with k = 25,000 and 30,000 large values in one
+    contiguous run: the candidates crowd into one or two select blocks'
+    ranges (more than one shared-memory staging round there) and into tiles
+    of more than 32 candidates (rescanned from the residual).  Three EF
+    steps; the streaming pass + select path, no rescan of the whole residual."""
+    n, k = 3_000_017, 25_000
+    rng = np.random.default_rng(77)
+    grads = []
+    for s in range(3):
+        g = rng.laplace(0, 1e-3, n).astype(np.float32)
+        a = 1_234_567 + 1000 * s
+        g[a:a + 30_000] = (rng.uniform(1.0, 2.0, 30_000) *
+                           np.where(rng.random(30_000) < 0.5, -1, 1)).astype(np.float32)
+        grads.append(g)
+    ws = _ws(n, k)
+    run_compress_steps(grads, LR, k, backend=1, ws=ws)
+    info = ef.topk_ef_path_info(ws)
+    assert info["fallback"] == 0 and info["kernels"] == 3, info
+
+
 def test_all_equal_magnitude():
     n, k = 150_000, 4321
     rng = np.random.default_rng(3)
