@@ -44,6 +44,10 @@ struct MergeSetupParams {
 __global__ void __launch_bounds__(MZ_THREADS)
 merge_setup_kernel(const MergeSetupParams p) {
     const int b = blockIdx.x, tid = threadIdx.x;
+    // the first round may be scheduled now (it waits for this grid); this
+    // grid waits for the kernel before it on the stream
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((uint32_t)b < p.validate_blocks) {
         const int64_t tot = (int64_t)p.P * p.k_in;
         bool bad = false;

@@ -1048,7 +1048,9 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     sp.ctrl = ctrl;
     sp.kernels = kernels;
     sp.zero_ptr = reinterpret_cast<uint4*>(w + L.zero_begin);
-    sp.zero_vec4 = (L.zero_end - L.zero_begin) / 16;
+    // the per-pair histograms and live counts serve only the merge + select
+    // kernels; the cluster kernel keeps its histograms in shared memory
+    sp.zero_vec4 = cluster_path ? 0 : (L.zero_end - L.zero_begin) / 16;
     sp.bad_words = bad;
     sp.sizes = sizes;
     sp.set_idx = set_idx;
@@ -1059,9 +1061,8 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     const int nz = (int)std::max<uint64_t>(
         1, std::min<uint64_t>(148, (sp.zero_vec4 + MZ_THREADS * 8 - 1) / (MZ_THREADS * 8)));
     trace_before(st, "merge_setup_kernel");
-    merge_setup_kernel<<<L.vblocks + nz, MZ_THREADS, 0, st>>>(sp);
+    cudaError_t e = launch_pdl(merge_setup_kernel, (int)(L.vblocks + nz), MZ_THREADS, st, sp);
     trace_after(st);
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
 
     const int G = std::min(SLOT_MAX, f.sms * f.selm_blocks);
