@@ -676,6 +676,9 @@ def run_ours(args):
             "config": wl.config(),
             "roofline": roof,
             "hbm_frac_whole_step": round(gbs / world / peak, 4),
+            "north_star_bar": {"judged_on": "whole call (hbm_frac_whole_step): setup, "
+                                            "streaming pass and select", "bar": 0.60,
+                               "met": bool(gbs / world / peak >= 0.60)},
             "gpu_launches": launches,
             "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / v[0], 5)}
                         for k, v in per_kernel.items()},
