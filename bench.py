@@ -94,18 +94,19 @@ def sources_sha():
     return h.hexdigest()
 
 
-def traffic_per_launch(kernel: str, n: int):
+def traffic_per_launch(kernel: str, workload: str):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
-    summary, scaled to n elements; None if absent or the kernel changed."""
+    summary, for the workload it was captured on only; None if absent, for
+    another workload, or if the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)[kernel]
     except (OSError, KeyError, ValueError):
         return None
-    if t.get("src_sha256") != sources_sha():
+    if t.get("src_sha256") != sources_sha() or t.get("bench_workload") != workload:
         return None
-    return float(t["dram_bytes"]) * n / float(t["n"])
+    return float(t["dram_bytes"])
 
 
 class ClockSampler:
@@ -633,7 +634,7 @@ def run_ours(args):
         roof = {"bound": "hbm", "kernel": wl.dominant, "achieved": round(ach, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
                 "peak_source": f"{peak_src} (hbm_gbs, burst copy)",
-                "traffic": traffic_per_launch(wl.dominant, wl.n) if hasattr(wl, "n") else None,
+                "traffic": traffic_per_launch(wl.dominant, args.workload),
                 "algorithmic_bytes_per_launch": wl.dominant_bytes,
                 "avg_launch_ms": round(avg, 5), "launches": len(dom)}
     per_kernel = {}

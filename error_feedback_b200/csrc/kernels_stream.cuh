@@ -156,8 +156,15 @@ __device__ __forceinline__ void stream_tile_record(const StreamParams& p, uint32
 // Each warp owns whole warp tiles, so warps never wait for one another; the
 // select kernel rebuilds the ordered candidate list from the records.  The loop
 // over full tiles of one tensor is kept small; everything else is out of line.
-template <bool VEC>
-__global__ void __launch_bounds__(K1_THREADS, 3)
+// MINB: resident blocks per SM the registers are sized for.  A single tensor
+// with a short candidate list runs 4 per SM (64 registers): the step of the
+// 25.6M-element workload at 0.1% and 0.01% density measured 1.2 to 2 us
+// faster, although the kernel alone is slower.  Everything else runs 3 per
+// SM (80 registers), which measured faster for a bucket (3.5 us on the
+// VGG-16 bucket), for long candidate lists (2 us at 1% density; 90 us on
+// 1.5e9 elements) and for the hard-threshold step (4 us).
+template <bool VEC, int MINB>
+__global__ void __launch_bounds__(K1_THREADS, MINB)
 stream_kernel(const __grid_constant__ StreamParams p) {
     __shared__ StreamShared S;
     const int tid = threadIdx.x;

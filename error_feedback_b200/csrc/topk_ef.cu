@@ -93,7 +93,9 @@ void trace_after(cudaStream_t st) {
 
 struct DevFacts {
     int sms = 0;
-    int k1_blocks = 0;       // resident stream_kernel blocks per SM
+    int k1_blocks = 0;       // resident stream_kernel<.., 3> blocks per SM (a bucket)
+    int k1_blocks1 = 0;      // resident stream_kernel<.., 4> blocks per SM (one tensor,
+                             // short candidate list)
     int selc_blocks = 0;     // resident select_kernel<CompressSrc> blocks per SM
     int selm_blocks = 0;     // resident select_kernel<MergeSrc> blocks per SM
     int fs_blocks = 0;       // resident flat_select_kernel blocks per SM
@@ -114,7 +116,12 @@ int device_facts(DevFacts* out) {
         DevFacts f;
         if ((e = cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail(e);
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.k1_blocks, stream_kernel<true>,
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.k1_blocks,
+                                                               stream_kernel<true, 3>,
+                                                               K1_THREADS, 0)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&f.k1_blocks1,
+                                                               stream_kernel<true, 4>,
                                                                K1_THREADS, 0)) != cudaSuccess)
             return cuda_fail(e);
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
@@ -136,7 +143,8 @@ int device_facts(DevFacts* out) {
         if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                  &f.sk_blocks, small_kernel, SK_THREADS, sizeof(SmallShared))) != cudaSuccess)
             return cuda_fail(e);
-        if (f.sms <= 0 || f.k1_blocks <= 0 || f.selc_blocks <= 0 || f.selm_blocks <= 0)
+        if (f.sms <= 0 || f.k1_blocks <= 0 || f.k1_blocks1 <= 0 || f.selc_blocks <= 0 ||
+            f.selm_blocks <= 0)
             return TOPK_EF_ERR_CUDA;
         g_facts[dev] = f;
         g_facts_ready[dev] = true;
@@ -350,7 +358,7 @@ cudaError_t launch_setup(const Group& g, const CLayout& L, char* ws, const float
 // programmatic serialisation); fills *sp for the select kernels.
 cudaError_t launch_stream(const Group& g, const CLayout& L, char* ws, const float* gg, float* rg,
                           float lr, cudaStream_t st, const DevFacts& f, StreamParams* sp_out,
-                          bool build_r1) {
+                          bool build_r1, bool four = false) {
     StreamParams sp;
     sp.grad = gg;
     sp.resid = rg;
@@ -368,12 +376,19 @@ cudaError_t launch_stream(const Group& g, const CLayout& L, char* ws, const floa
                 : nullptr;
     *sp_out = sp;
     const bool vec = ((uintptr_t)gg % 16 == 0) && ((uintptr_t)rg % 16 == 0);
+    const bool one = four && g.plans.size() == 1;
     const int64_t warps_needed = L.num_wt;
+    const int per_sm = one ? f.k1_blocks1 : f.k1_blocks;
     const int g1 = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div64(warps_needed, K1_THREADS / 32),
-                                                               (int64_t)f.sms * f.k1_blocks));
+                                                               (int64_t)f.sms * per_sm));
     trace_before(st, "stream_kernel");
-    cudaError_t e = vec ? launch_pdl(stream_kernel<true>, g1, K1_THREADS, st, sp)
-                        : launch_pdl(stream_kernel<false>, g1, K1_THREADS, st, sp);
+    cudaError_t e;
+    if (one)
+        e = vec ? launch_pdl(stream_kernel<true, 4>, g1, K1_THREADS, st, sp)
+                : launch_pdl(stream_kernel<false, 4>, g1, K1_THREADS, st, sp);
+    else
+        e = vec ? launch_pdl(stream_kernel<true, 3>, g1, K1_THREADS, st, sp)
+                : launch_pdl(stream_kernel<false, 3>, g1, K1_THREADS, st, sp);
     trace_after(st);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e;
@@ -495,7 +510,9 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     // would pay more in the streaming pass than the barrier it saves costs)
     const bool build_r1 = T == 1 && (flat || L.cap <= ((int64_t)1 << 19));
     StreamParams sp;
-    if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp, build_r1)) != cudaSuccess)
+    // the flat select with a short candidate list: 4 streaming blocks per SM
+    const bool four = flat && L.cap <= ((int64_t)1 << 19);
+    if ((e = launch_stream(g, L, ws, gg, rg, lr, st, f, &sp, build_r1, four)) != cudaSuccess)
         return cuda_fail(e);
     if (flat_skip) return TOPK_EF_OK;
     Ctrl* ctrl = sp.ctrl;
