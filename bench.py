@@ -184,6 +184,16 @@ def l2_note(flush: bool, input_bytes: int) -> str:
             f"126 MB L2; steps run back to back")
 
 
+def hbm_bar(wl, frac):
+    """The 60%-of-HBM bar set for the Top-k + EF compress of n >= 25.6M
+    elements, judged on the whole call; other workloads are not held to it."""
+    if isinstance(wl, (FlatCompress, BatchedCompress)) and wl.n >= datagen.RESNET50_N:
+        return {"judged_on": "whole call (hbm_frac_whole_step): setup, streaming pass "
+                             "and select", "bar": 0.60, "met": bool(frac >= 0.60)}
+    return {"applies": False,
+            "why": "the bar is set for the Top-k + EF compress of n >= 25.6M elements"}
+
+
 class FlatCompress:
     """One EF step of topk_ef_compress on a flat gradient."""
 
@@ -677,9 +687,7 @@ def run_ours(args):
             "config": wl.config(),
             "roofline": roof,
             "hbm_frac_whole_step": round(gbs / world / peak, 4),
-            "hbm_bar": {"judged_on": "whole call (hbm_frac_whole_step): setup, "
-                                            "streaming pass and select", "bar": 0.60,
-                               "met": bool(gbs / world / peak >= 0.60)},
+            "hbm_bar": hbm_bar(wl, gbs / world / peak),
             "gpu_launches": launches,
             "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / v[0], 5)}
                         for k, v in per_kernel.items()},
