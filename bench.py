@@ -33,7 +33,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -48,7 +47,7 @@ METRIC = "Top-k+EF compress GB/s & elems/s at n=25.6M, density 0.1% (% of HBM pe
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20       # B200 L2; step inputs above this run back to back
-TRACE_EVERY = 8            # timed region: events around every 8th dominant launch
+TRACE_BRACKETS = 4         # timed region: events around at most this many dominant launches
 LR = np.float32(0.1)
 POOL = 4          # distinct gradients cycled through the steps
 KERNEL_SOURCES = ["error_feedback_b200/csrc/kernels_stream.cuh",
@@ -109,55 +108,129 @@ def traffic_per_launch(kernel: str, workload: str):
     return float(t["dram_bytes"])
 
 
-class ClockSampler:
-    """Polls SM clock and throttle reasons through NVML while running."""
+_SAMPLER_CHILD = r"""
+import select, sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+period = float(sys.argv[2])
+reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+           or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+rows = []
+while True:
+    t = time.monotonic()
+    rows.append((t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(reasons(h))))
+    if len(rows) == 1:
+        print("ready", flush=True)
+    r, _, _ = select.select([sys.stdin], [], [], period)
+    if r and not sys.stdin.read(1):
+        break
+for t, m, rs in rows:
+    print(t, m, rs)
+"""
 
-    def __init__(self, torch_dev: int, period_s: float = 0.005):
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while running.
+
+    The polling runs in a child process: a thread of this process would take
+    the interpreter lock from the loop that launches the timed steps and
+    delay them.  Samples are stamped with the host's monotonic clock, and
+    only those taken between entry and exit are kept."""
+
+    def __init__(self, torch_dev: int, period_s: float = 0.0005, uuid: str | None = None):
         self.samples = []
         self.max_mhz = None
         self.err = None
         self.period = period_s
-        self._stop = threading.Event()
-        self._thr = None
+        self.proc = None
+        self.uuid = uuid
+        if uuid is None:
+            try:
+                import torch
+                u = str(torch.cuda.get_device_properties(torch_dev).uuid)
+                self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+            except Exception as e:  # noqa: BLE001
+                self.err = f"{type(e).__name__}: {e}"
+
+    def start(self):
+        """Start polling (a child process: its start-up takes a fraction of a
+        second, so start it before the warm-up, not just before timing)."""
+        import select
+        import subprocess
+        self.t0 = time.monotonic()
+        if self.uuid is None:
+            return self
         try:
-            import pynvml
-            import torch
-            pynvml.nvmlInit()
-            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
-            if not uuid.startswith("GPU-"):
-                uuid = "GPU-" + uuid
-            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
-            self.nv = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", _SAMPLER_CHILD, self.uuid, str(self.period)],
+                stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.PIPE)
+            # unbuffered reads of the child's first lines (a buffered reader
+            # would swallow lines that select() then never reports)
+            fd = self.proc.stdout.fileno()
+            head = b""
+            deadline = time.monotonic() + 60
+            while b"ready\n" not in head:
+                left = deadline - time.monotonic()
+                if left <= 0 or not select.select([fd], [], [], left)[0]:
+                    raise RuntimeError("NVML sampler did not start")
+                chunk = os.read(fd, 4096)
+                if not chunk:
+                    raise RuntimeError("NVML sampler exited: "
+                                       + self.proc.stderr.read().decode(errors="replace")[-300:])
+                head += chunk
+            for line in head.decode().splitlines():
+                if line.startswith("max "):
+                    self.max_mhz = int(line.split()[1])
         except Exception as e:  # noqa: BLE001
             self.err = f"{type(e).__name__}: {e}"
-            self.h = None
-
-    def _run(self):
-        nv = self.nv
-        while not self._stop.is_set():
-            try:
-                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
-                try:
-                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                except AttributeError:
-                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                self.samples.append((mhz, int(rs)))
-            except Exception as e:  # noqa: BLE001
-                self.err = str(e)
-                return
-            time.sleep(self.period)
-
-    def __enter__(self):
-        if self.h is not None:
-            self._thr = threading.Thread(target=self._run, daemon=True)
-            self._thr.start()
+            self._end()
+        self.t0 = time.monotonic()
         return self
 
+    def mark(self):
+        """Keep only the samples taken from now on."""
+        self.t0 = time.monotonic()
+
+    def __enter__(self):
+        return self.start()
+
+    def _end(self):
+        import subprocess
+        if self.proc is None:
+            return ""
+        out = b""
+        try:
+            out, _ = self.proc.communicate(input=b"", timeout=30)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.proc.communicate()
+            self.err = "NVML sampler did not stop"
+        self.proc = None
+        return out.decode(errors="replace")
+
     def __exit__(self, *a):
-        self._stop.set()
-        if self._thr:
-            self._thr.join()
+        self.stop()
+
+    def stop(self):
+        """Stop polling; keeps the samples taken since start() or mark()."""
+        t1 = time.monotonic()
+        rows = []
+        for line in self._end().splitlines():
+            f = line.split()
+            if len(f) == 3:
+                try:
+                    rows.append((float(f[0]), int(f[1]), int(f[2])))
+                except ValueError:
+                    pass
+        inside = [(m, r) for t, m, r in rows if self.t0 <= t <= t1]
+        if not inside and rows:
+            # a region shorter than the polling interval: the nearest sample
+            t_mid = 0.5 * (self.t0 + t1)
+            _, m, r = min(rows, key=lambda x: abs(x[0] - t_mid))
+            inside = [(m, r)]
+        self.samples = inside
 
     def summary(self):
         names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -576,6 +649,9 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    # clock polling starts before the warm-up, so that its start-up does not
+    # leave the GPU idle just before the timed region
+    clk = ClockSampler(local).start()
     for w in range(args.warmup):
         if wl.flush:
             flush.fill_(float(w))
@@ -583,6 +659,7 @@ def run_ours(args):
     barrier()
     st = wl.status()
     if st != 0:
+        clk.stop()
         raise SystemExit(f"device status after warm-up: {ef.status_string(st)}")
     if hasattr(wl, "after_warmup"):
         wl.after_warmup()
@@ -601,26 +678,32 @@ def run_ours(args):
 
     # timed region: K steps; inputs larger than L2 run back to back, smaller
     # ones get an L2 flush before each step (outside the timed intervals).
-    # Only the dominant kernel is bracketed by events, every TRACE_EVERY-th
-    # launch of it, so that the launches keep overlapping as they do untraced.
-    ef.topk_ef_trace_enable(True, only=wl.dominant, every=TRACE_EVERY)
+    # Only the dominant kernel is bracketed by events, and only a few of its
+    # launches spread over the region (one per ten, at most TRACE_BRACKETS):
+    # events between two launches stop the second from starting early, so
+    # every bracket slows the step it falls in.
+    dom_launches = sum(1 for name, _ in trace_all if name == wl.dominant) * args.steps // nt
+    brackets = min(TRACE_BRACKETS, max(1, dom_launches // 10))
+    every = max(1, -(-dom_launches // brackets))
+    ef.topk_ef_trace_enable(True, only=wl.dominant, every=every)
     barrier()
-    with ClockSampler(local) as clk:
-        if wl.flush:
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
-            for i in range(args.steps):
-                flush.fill_(float(i))
-                ev[i][0].record(stream)
-                wl.step(args.warmup + i)
-                ev[i][1].record(stream)
-        else:
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))]
-            ev[0][0].record(stream)
-            for i in range(args.steps):
-                wl.step(args.warmup + i)
-            ev[0][1].record(stream)
-        barrier()
+    clk.mark()
+    if wl.flush:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            wl.step(args.warmup + i)
+            ev[i][1].record(stream)
+    else:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))]
+        ev[0][0].record(stream)
+        for i in range(args.steps):
+            wl.step(args.warmup + i)
+        ev[0][1].record(stream)
+    barrier()
+    clk.stop()
     trace = ef.topk_ef_trace_read()
     ef.topk_ef_trace_enable(False)
     st = wl.status()
