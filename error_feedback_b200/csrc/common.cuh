@@ -63,7 +63,10 @@ struct Ctrl {
     uint32_t r2_path;       // compress: a tensor's k-th bin was too full for its entry list
     uint32_t merge_bar[32]; // grid barrier counters, one per merge round
     uint32_t stall;         // test hook: extra arrivals the flat select's barrier waits for
-    uint32_t pad1[5];
+    uint32_t path_small;    // SK_PATH_TAG: the last call was small_kernel's (status below)
+    uint64_t sk_status;     // small_kernel: call tag (high half) and ST_* bits
+    uint32_t sk_tag;        // small_kernel: the last call's tag (low half)
+    uint32_t pad1;
     uint64_t t_phase[8];    // select kernel: globaltimer at each phase (block 0)
     uint64_t t_span[8];     // globaltimer over all blocks (diagnostics): the first
                             // block of a kernel stores ~t (atomicMax of the

@@ -4,8 +4,7 @@
 //   topk_ef_compress / _batched:  setup_kernel -> stream_kernel -> select kernel
 //                                 (flat_select_kernel for a single tensor,
 //                                 select_kernel<CompressSrc> for a bucket);
-//                                 a single small tensor: setup_kernel ->
-//                                 small_kernel
+//                                 a single small tensor: small_kernel alone
 //   gtopk_merge:                  merge_setup_kernel -> (merge_round_kernel ->
 //                                 select_kernel) per tournament round
 //
@@ -15,9 +14,11 @@
 
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <random>
 #include <string>
 #include <vector>
 
@@ -223,7 +224,7 @@ TensorPlan plan_tensor(int64_t off, int64_t n, int64_t k, int64_t out_base) {
 // Workspace layout of one compress group (<= TCAP_LARGE tensors).
 struct CLayout {
     size_t ctrl, meta, hint, zero_begin, cand_start, ent_cnt, agg, hist, zero_end, wt_count, wt_off,
-        ent, slots, cand_idx, cand_val, total;
+        ent, slots, cand_idx, cand_val, sk_sync, sk_idx, sk_val, total;
     int64_t cap;
     uint32_t num_wt;
 };
@@ -264,6 +265,17 @@ CLayout compress_layout(int64_t N, const std::vector<TensorPlan>& plans) {
     o = align_up(o + (size_t)cap * sizeof(uint32_t));
     L.cand_val = o;
     o = align_up(o + (size_t)cap * sizeof(float));
+    // a single tensor small enough for small_kernel: its arrival words and
+    // its candidate regions (one per block, at the block's slice)
+    L.sk_sync = L.sk_idx = L.sk_val = 0;
+    if (T == 1 && N > 0 && N <= SK_N_MAX) {
+        L.sk_sync = o;
+        o = align_up(o + sizeof(SkSync));
+        L.sk_idx = o;
+        o = align_up(o + (size_t)N * sizeof(uint32_t));
+        L.sk_val = o;
+        o = align_up(o + (size_t)N * sizeof(float));
+    }
     L.total = o;
     return L;
 }
@@ -434,6 +446,19 @@ uint64_t hint_tag_of(const float* resid, int64_t n, uint32_t k, float lr) {
     return h ? h : 1;
 }
 
+// A number distinct for every small_kernel launch of this process (a counter
+// mixed with a per-process random start).  The kernel mixes it with the
+// workspace's own call counter, so that a replayed graph differs too.
+uint64_t next_call_tag() {
+    static std::atomic<uint64_t> ctr{0};
+    static const uint64_t start = [] {
+        std::random_device rd;
+        const uint64_t t = (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
+        return ((uint64_t)rd() << 32) ^ (uint64_t)rd() ^ (t * 0x9E3779B97F4A7C15ull);
+    }();
+    return start + 0xD1B54A32D192ED03ull * (ctr.fetch_add(1) + 1);
+}
+
 int compress_group(const Group& g, const float* grad, float* resid, float lr, int32_t* out_idx,
                    float* out_val, char* ws, cudaStream_t st, const DevFacts& f, int flags) {
     const CLayout L = compress_layout(g.N, g.plans);
@@ -448,16 +473,11 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
     // block; a bucket (or a huge tensor) takes the segmented select.
     const int G_flat = std::min(SLOT_MAX, f.sms);
     // A single tensor that one wave of blocks holds in shared memory takes
-    // small_kernel (no prefilter, no separate select)
-    const int sm_cap = std::min(SLOT_MAX, f.sms);
+    // small_kernel alone: one launch, no setup
+    const int sm_cap = std::min(SK_GRID_MAX, f.sms);
     const bool small = T == 1 && f.sk_blocks >= 1 && g.N > 0 && g.plans[0].k > 0 &&
-                       !force_dense && g.N <= (int64_t)sm_cap * SK_MAX;
+                       !force_dense && L.sk_sync != 0 && g.N <= (int64_t)sm_cap * SK_MAX;
     if (small) {
-        trace_before(st, "setup_kernel");
-        cudaError_t e = launch_setup<TCAP_SMALL>(g, L, ws, grad + g.base, resid + g.base, lr,
-                                                 true, 2u, st, nullptr, 0, stall);
-        trace_after(st);
-        if (e != cudaSuccess) return cuda_fail(e);
         const int G = (int)std::max<int64_t>(1, std::min<int64_t>(sm_cap,
                                                    ceil_div64(g.N, SK_MIN_PER_BLOCK)));
         SmallParams kp;
@@ -476,6 +496,17 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
         kp.ent = reinterpret_cast<uint32_t*>(ws + L.ent);
         kp.ent_cnt = reinterpret_cast<uint32_t*>(ws + L.ent_cnt);
         kp.slots = reinterpret_cast<Slot*>(ws + L.slots);
+        kp.sync = reinterpret_cast<SkSync*>(ws + L.sk_sync);
+        kp.cand_idx = reinterpret_cast<uint32_t*>(ws + L.sk_idx);
+        kp.cand_val = reinterpret_cast<float*>(ws + L.sk_val);
+        kp.hint = reinterpret_cast<Hint*>(ws + L.hint);
+        // the threshold hint: for a k that block 0 can select from alone, and
+        // tagged apart from the flat path's hint
+        kp.hint_tag = kp.k <= SK_HINT_KMAX && !force_t0
+                          ? (hint_tag_of(rg, g.N, kp.k, lr) ^ 0x5A5A5A5A00000000ull) | 1ull : 0;
+        kp.call_tag = next_call_tag();
+        kp.force_t0 = force_t0 ? 1u : 0u;
+        kp.stall = stall;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(G);
         cfg.blockDim = dim3(SK_THREADS);
@@ -487,7 +518,7 @@ int compress_group(const Group& g, const float* grad, float* resid, float lr, in
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         trace_before(st, "small_kernel");
-        e = cudaLaunchKernelEx(&cfg, small_kernel, kp);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, small_kernel, kp);
         trace_after(st);
         return e == cudaSuccess ? TOPK_EF_OK : cuda_fail(e);
     }
@@ -1204,10 +1235,15 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
 int topk_ef_last_device_status(const void* ws, void* stream) {
     if (!ws) return TOPK_EF_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    uint32_t s = 0;
-    cudaError_t e = cudaMemcpyAsync(&s, ws, sizeof(s), cudaMemcpyDeviceToHost, st);
+    Ctrl c;
+    cudaError_t e = cudaMemcpyAsync(&c, ws, sizeof(c), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e);
+    // small_kernel records its errors with the call's tag (nothing clears the
+    // word before a call); every other path clears the control block first
+    const uint32_t s = c.path_small == SK_PATH_TAG
+                           ? ((uint32_t)(c.sk_status >> 32) == c.sk_tag ? (uint32_t)c.sk_status : 0u)
+                           : c.status;
     if (s & ST_TIMEOUT) return TOPK_EF_ERR_DEVICE_TIMEOUT;
     if (s & ST_BAD_INPUT) return TOPK_EF_ERR_BAD_INPUT;
     if (s & ST_INCONSISTENT) return TOPK_EF_ERR_INTERNAL;

@@ -59,21 +59,30 @@ def assert_same_step(step, gi, gv, gres, oi, ov, ores):
                              f"gpu {gres[bad[0]]!r} oracle {ores[bad[0]]!r}")
 
 
-def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=None, n=None):
+def run_compress_steps(grads, lr, k, res0=None, backend=0, offset_elems=0, ws=None, n=None,
+                       paths=None, zero_between=False):
     """EF steps on the GPU and in the oracle; every step compared.
     grads: float32 arrays, one per step (a list, or any iterable when n is
-    given, so that full-size sequences need not be held at once).  Returns
-    the GPU residual."""
+    given, so that full-size sequences need not be held at once).
+    paths: a list that receives topk_ef_path_info after every step (needs
+    ws).  zero_between: both residuals are set to +0 before every step after
+    the first (the caller owns the residual; the workspace, and with it the
+    previous call's threshold hint, is kept).  Returns the GPU residual."""
     o = oracle.get()
     if n is None:
         n = grads[0].size
     ores = np.zeros(n, np.float32) if res0 is None else res0.copy()
     dres = to_dev(ores, offset_elems)
     for s, g in enumerate(grads):
+        if zero_between and s > 0:
+            ores[:] = 0
+            dres.zero_()
         dg = to_dev(g, offset_elems)
         gi, gv = ef.topk_ef_compress(dg, dres, lr, k, ws=ws)
         st = ef.topk_ef_last_device_status(ws) if ws is not None else 0
         assert st == 0, ef.status_string(st)
+        if paths is not None:
+            paths.append(ef.topk_ef_path_info(ws))
         oi, ov = o.compress(g, ores, lr, k, backend)
         assert_same_step(s, gi, gv, dres, oi, ov, ores)
     return dres

@@ -25,8 +25,198 @@ def test_flat_normal_1m():
     ws = _ws(n, k)
     run_compress_steps(grads, LR, k, ws=ws)
     info = ef.topk_ef_path_info(ws)
-    # a tensor this small takes the one-kernel path (setup + small_kernel)
-    assert info["fallback"] == 0 and info["kernels"] == 2, info
+    # a tensor this small takes one launch (small_kernel, no setup)
+    assert info["kernels"] == 1, info
+
+
+# Small tensors (one wave of blocks): small_kernel lists the elements that
+# reach the previous call's threshold and, when that list decides the top k
+# (at least k and at most 8,192 of them), every block selects from that list
+# after one exchange ("fallback" 0); otherwise every block runs the exact
+# two-exchange select ("fallback" 1).  Both must give the oracle's answer bit for bit.
+SK_CAP1 = 8192
+
+
+def test_small_bench_sequence():
+    """The 1M flat workload's own sequence: one residual through 32 EF steps
+    whose gradients cycle through a pool of 4, as the benchmark runs it.
+    Early steps widen |acc| too fast for the previous threshold; later ones
+    take it."""
+    n, k = 1 << 20, 1048
+    pool = [datagen.flat_normal(s) for s in range(4)]
+    ws = _ws(n, k)
+    paths = []
+    run_compress_steps([pool[i % 4] for i in range(32)], LR, k, ws=ws, paths=paths)
+    assert paths[0]["fallback"] == 1            # no threshold yet
+    late = [p["fallback"] for p in paths[16:]]
+    assert late.count(0) >= 14, [(p["fallback"], p["candidates"]) for p in paths]
+    for p in paths:
+        assert p["kernels"] == 1
+        assert p["fallback"] == 1 or k <= p["candidates"] <= SK_CAP1, p
+
+
+def test_small_threshold_misses_both_ways():
+    """The threshold hint stays valid while the caller zeroes the residual,
+    so acc = lr * grad: steady gradients take it; a step with gradients 1000x
+    smaller leaves fewer than k above it, the next step at full scale puts
+    almost every element above the small step's threshold; both fall back to
+    the exact path and the step after takes the hint again."""
+    n, k = 1 << 20, 1048
+    rng = np.random.default_rng(5)
+    scale = [1, 1, 1, 1, 1e-3, 1, 1, 1]
+    grads = [(rng.standard_normal(n) * s).astype(np.float32) for s in scale]
+    ws = _ws(n, k)
+    paths = []
+    run_compress_steps(grads, LR, k, ws=ws, paths=paths, zero_between=True)
+    got = [p["fallback"] for p in paths]
+    assert got == [1, 0, 0, 0, 1, 1, 0, 0], [(p["fallback"], p["candidates"]) for p in paths]
+    assert paths[4]["candidates"] < k and paths[5]["candidates"] > SK_CAP1
+
+
+def test_small_hint_ties():
+    """3,000 entries of magnitude exactly 1.0 among values below 0.4: the k-th
+    key is shared by all of them, the threshold path sees exactly those
+    3,000 and must keep the k lowest indices."""
+    n, k = 100_000, 1000
+    rng = np.random.default_rng(8)
+    grads = []
+    for _ in range(4):
+        g = rng.uniform(-0.4, 0.4, n).astype(np.float32)
+        pos = rng.choice(n, 3000, replace=False)
+        g[pos] = rng.choice(np.array([1.0, -1.0], np.float32), 3000)
+        grads.append(g)
+    ws = _ws(n, k)
+    paths = []
+    run_compress_steps(grads, np.float32(1.0), k, ws=ws, paths=paths, zero_between=True)
+    assert [p["fallback"] for p in paths] == [1, 0, 0, 0], paths
+    assert all(p["candidates"] == 3000 for p in paths[1:]), paths
+
+
+@pytest.mark.parametrize("k,paths", [(200, [1, 0, 0, 0]), (50, None)])
+def test_small_hint_special_values(k, paths):
+    """NaN, +-Inf and -0 among small normal values: the NaNs rank first (one
+    key above +Inf).  With k = 200 the k-th key is a normal value and the
+    threshold path counts the specials in its open top bin; with k = 50 the
+    infinities share the k-th key, far above the threshold's bins, and the
+    lower indices must win (the exact path takes that case)."""
+    n = 50_000
+    rng = np.random.default_rng(9)
+    grads = []
+    for _ in range(4):
+        g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+        pos = rng.choice(n, 100, replace=False)
+        g[pos[:30]] = np.float32(np.nan)
+        g[pos[30:50]] = np.float32(np.inf)
+        g[pos[50:70]] = np.float32(-np.inf)
+        g[pos[70:]] = np.float32(-0.0)
+        grads.append(g)
+    ws = _ws(n, k)
+    got = []
+    run_compress_steps(grads, np.float32(1.0), k, ws=ws, paths=got, zero_between=True)
+    if paths is not None:
+        assert [p["fallback"] for p in got] == paths, got
+
+
+@pytest.mark.parametrize("offset", [1, 2, 3])
+def test_small_hint_unaligned(offset):
+    """grad/residual not 16-byte aligned on the threshold path."""
+    n, k = 300_007, 301
+    rng = np.random.default_rng(20 + offset)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(4)]
+    ws = _ws(n, k)
+    paths = []
+    run_compress_steps(grads, LR, k, offset_elems=offset, ws=ws, paths=paths, zero_between=True)
+    assert [p["fallback"] for p in paths][1:] == [0, 0, 0], paths
+
+
+@pytest.mark.parametrize("n,k,path", [(5000, 100, 0), (8192, 8192, 0), (8192, 5, 0),
+                                      (8193, 5, 1), (20_000, 100, 1)])
+def test_small_threshold_zero(n, k, path):
+    """Test flag bit 1 (threshold 0): every element is a candidate, so a
+    tensor of at most 8,192 elements takes the threshold path over its whole
+    key range and a larger one the exact path."""
+    rng = np.random.default_rng(n)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(2)]
+    ws = _ws(n, k)
+    paths = []
+    old = ef.topk_ef_set_test_flags(2)
+    try:
+        run_compress_steps(grads, LR, k, ws=ws, paths=paths)
+    finally:
+        ef.topk_ef_set_test_flags(old)
+    assert [p["fallback"] for p in paths] == [path, path], paths
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, 0xA5])
+def test_small_workspace_contents(fill):
+    """The kernel needs no cleared state: a workspace of zeros, of ones or of
+    a pattern gives exact results from the first call on."""
+    n, k = 1 << 20, 1048
+    ws = torch.full((ef.topk_ef_workspace_bytes(n, k),), fill, dtype=torch.uint8, device="cuda")
+    rng = np.random.default_rng(fill)
+    grads = [rng.standard_normal(n).astype(np.float32) for _ in range(3)]
+    run_compress_steps(grads, LR, k, ws=ws, zero_between=True)
+
+
+def test_small_two_residuals_one_workspace():
+    """Two tensors' steps interleaved on one workspace: each call's hint is
+    tagged with its residual, so neither takes the other's threshold."""
+    import oracle
+    o = oracle.get()
+    n, k = 400_000, 400
+    rng = np.random.default_rng(31)
+    ws = _ws(n, k)
+    ores = [np.zeros(n, np.float32), np.zeros(n, np.float32)]
+    dres = [torch.zeros(n, dtype=torch.float32, device="cuda") for _ in range(2)]
+    for step in range(6):
+        t = step % 2
+        g = (rng.standard_normal(n) * (1.0 if t == 0 else 1e-4)).astype(np.float32)
+        gi, gv = ef.topk_ef_compress(to_dev(g), dres[t], LR, k, ws=ws)
+        assert ef.topk_ef_last_device_status(ws) == 0
+        oi, ov = o.compress(g, ores[t], LR, k, 0)
+        from gpu_util import assert_same_step
+        assert_same_step(step, gi, gv, dres[t], oi, ov, ores[t])
+
+
+def test_small_graph_replay():
+    """One compress call captured in a CUDA graph and replayed with new
+    gradients: every replay is exact (the launch parameters repeat, the
+    workspace's call counter keeps the replays apart)."""
+    import oracle
+    o = oracle.get()
+    n, k = 1 << 20, 1048
+    pool = [datagen.flat_normal(s) for s in range(4)]
+    ws = _ws(n, k)
+    g = torch.empty(n, dtype=torch.float32, device="cuda")
+    dres = torch.zeros(n, dtype=torch.float32, device="cuda")
+    oi_ = torch.empty(k, dtype=torch.int32, device="cuda")
+    ov_ = torch.empty(k, dtype=torch.float32, device="cuda")
+    ores = np.zeros(n, np.float32)
+    # two eager steps (the library's one-time device queries happen here)
+    for step in range(2):
+        g.copy_(torch.from_numpy(pool[step]))
+        ef.topk_ef_compress(g, dres, LR, k, oi_, ov_, ws=ws)
+        oi, ov = o.compress(pool[step], ores, LR, k, 0)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            ef.topk_ef_compress(g, dres, LR, k, oi_, ov_, ws=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    paths = []
+    from gpu_util import assert_same_step
+    for step in range(2, 14):
+        g.copy_(torch.from_numpy(pool[step % 4]))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert ef.topk_ef_last_device_status(ws) == 0
+        paths.append(ef.topk_ef_path_info(ws)["fallback"])
+        oi, ov = o.compress(pool[step % 4], ores, LR, k, 0)
+        assert_same_step(step, oi_, ov_, dres, oi, ov, ores)
+    del graph
+    assert 0 in paths, paths
 
 
 @pytest.mark.parametrize("n,k", [
