@@ -94,12 +94,12 @@ __device__ __forceinline__ uint64_t sk_arm(uint64_t seq) {
 
 struct SmallShared {
     float acc[SK_MAX];          // this block's acc
-    uint32_t own[SK_MAX];       // threshold path: slice positions of its candidates
+    uint32_t own[SK_CAP1];      // threshold path: slice positions of its candidates
     uint32_t hist[SK_BINS];     // threshold path: pass 1 [0, 4096), pass 2 above
-    uint8_t blk[SK_CAP1];       // threshold path: the block of each candidate
+    uint32_t ckey[SK_CAP1];     // threshold path: every candidate's key, index order
     uint64_t scan[33];
     uint32_t red[33];
-    FindResult fr;
+    FindResult fr, fr2;
     uint32_t pre;
     int flag;
     uint32_t pre_blk[SK_GRID_MAX + 1];  // candidates of the blocks before
@@ -262,6 +262,39 @@ __device__ __forceinline__ void sk_emit_ordered(uint32_t cnt, uint32_t gt0, uint
     __syncthreads();
 }
 
+// block_find_bin for two ranks with one scan (r1 -> *o1, r2 -> *o2).
+__device__ __forceinline__ void sk_find_two(const uint32_t* h, int nb, uint32_t r1, uint32_t r2,
+                                            uint32_t* s_red, FindResult* o1, FindResult* o2) {
+    const int t = threadIdx.x;
+    const int per = nb / (int)blockDim.x;
+    const int hi = nb - t * per;   // thread 0 owns the top bins
+    const int lo = hi - per;
+    uint32_t sum = 0;
+    for (int i = 0; i < per; ++i) sum += h[lo + ((i + t) & (per - 1))];
+    if (t == 0) o1->ok = o2->ok = 0;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(sum, s_red, &tot);
+    for (int w = 0; w < 2; ++w) {
+        const uint32_t rem = w == 0 ? r1 : r2;
+        FindResult* out = w == 0 ? o1 : o2;
+        if (ex < rem && ex + sum >= rem) {
+            uint32_t run = ex;
+            for (int b = hi - 1; b >= lo; --b) {
+                const uint32_t cnt = h[b];
+                if (run + cnt >= rem) {
+                    out->bin = (uint32_t)b;
+                    out->above = run;
+                    out->cnt = cnt;
+                    out->ok = 1;
+                    break;
+                }
+                run += cnt;
+            }
+        }
+    }
+    __syncthreads();
+}
+
 // Rank of the element whose bin sets the next call's threshold: above the
 // k-th, so that the next call's k-th key may be a little lower and still
 // pass, and low enough that the growth of |acc| under error feedback keeps
@@ -384,8 +417,8 @@ __device__ __noinline__ uint32_t sk_crowded(const SmallParams& p, SmallShared& K
 }
 
 // Threshold path, in every block: the E candidates of the G blocks' regions
-// (every element with key >= T0) decide the top k.  Each thread loads the
-// keys of positions tid + 512 u (index order) into registers and counts them
+// (every element with key >= T0) decide the top k.  Warp w gathers the keys
+// of blocks w, w + 16, ... into shared memory in index order and counts them
 // in SK_RBINS bins of (key - T0) >> sh, the top one open above; the k-th key
 // T and the tie quota q follow from those bins and the sh bits below (in two
 // steps above 12 bits).  Writes T, q and this block's counts of earlier
@@ -396,47 +429,63 @@ __device__ __noinline__ uint32_t sk_crowded(const SmallParams& p, SmallShared& K
 __device__ __forceinline__ bool sk_threshold_select(const SmallParams& p, SmallShared& K, int G,
                                                     int64_t per, uint32_t E, uint32_t T0,
                                                     uint32_t sh, uint32_t* out) {
-    constexpr int U = (int)(SK_CAP1 / SK_THREADS);     // keys per thread at most
     const int tid = threadIdx.x, c = blockIdx.x;
     const uint32_t k = p.k;
+    const uint32_t lane = lane_id(), w = warp_id();
+    constexpr int NW = SK_THREADS / 32;
+    constexpr int R = (SK_GRID_MAX + NW - 1) / NW;      // blocks per warp at most
     uint32_t* h1 = K.hist;
     uint32_t* h2 = K.hist + SK_RBINS;
-    // ---- the block each candidate position belongs to
-    if (tid < G)
-        for (uint32_t q = K.pre_blk[tid]; q < K.pre_blk[tid + 1]; ++q) K.blk[q] = (uint8_t)tid;
-    __syncthreads();
-    // ---- keys into registers, all loads first; pass 1
-    uint32_t key[U];
+    // ---- keys in index order: warp w takes blocks w, w + 16, ...; the first
+    // 64 candidates of each block all loaded at once, the rest after
+    {
+        float v[2][R];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint32_t q = (uint32_t)tid + (uint32_t)u * SK_THREADS;
-        key[u] = 0;
-        if (q < E) {
-            const int j = K.blk[q];
-            const int64_t at = min((int64_t)j * per, p.n) + (int64_t)(q - K.pre_blk[j]);
-            key[u] = __float_as_uint(__ldcg(p.cand_val + at));   // written by other blocks
+        for (int r = 0; r < R; ++r) {
+            const int j = (int)w + r * NW;
+            if (j < G) {
+                const uint32_t cnt = K.pre_blk[j + 1] - K.pre_blk[j];
+                const float* src = p.cand_val + min((int64_t)j * per, p.n);   // other blocks'
+                if (lane < cnt) v[0][r] = __ldcg(src + lane);
+                if (32 + lane < cnt) v[1][r] = __ldcg(src + 32 + lane);
+            }
         }
-    }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint32_t q = (uint32_t)tid + (uint32_t)u * SK_THREADS;
-        if (q < E) {
-            key[u] = key_of(__uint_as_float(key[u]));
-            atomicAdd(&h1[min((key[u] - T0) >> sh, (uint32_t)(SK_RBINS - 1))], 1u);
+        for (int r = 0; r < R; ++r) {
+            const int j = (int)w + r * NW;
+            if (j < G) {
+                const uint32_t a = K.pre_blk[j], cnt = K.pre_blk[j + 1] - a;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (32u * h + lane < cnt) {
+                        const uint32_t key = key_of(v[h][r]);
+                        K.ckey[a + 32u * h + lane] = key;
+                        atomicAdd(&h1[min((key - T0) >> sh, (uint32_t)(SK_RBINS - 1))], 1u);
+                    }
+                }
+            }
+        }
+        for (int j = (int)w; j < G; j += NW) {
+            const uint32_t a = K.pre_blk[j], cnt = K.pre_blk[j + 1] - a;
+            const int64_t base = min((int64_t)j * per, p.n);
+            for (uint32_t i = 64 + lane; i < cnt; i += 32) {
+                const uint32_t key = key_of(__ldcg(p.cand_val + base + i));
+                K.ckey[a + i] = key;
+                atomicAdd(&h1[min((key - T0) >> sh, (uint32_t)(SK_RBINS - 1))], 1u);
+            }
         }
     }
     __syncthreads();
     mark_phase(p.ctrl, 4);
+    // ---- pass 1: the k-th key's bin (block 0: also the bin of the hint's rank)
     uint32_t hb = NO_KEY;
-    if (c == 0 && p.hint_tag != 0) {
-        const uint32_t rh = sk_hint_rank(k);
-        if (rh <= E) {
-            block_find_bin(h1, SK_RBINS, rh, K.red, &K.fr);
-            if (K.fr.ok) hb = K.fr.bin;
-        }
-        __syncthreads();
+    const uint32_t rh = sk_hint_rank(k);
+    if (c == 0 && p.hint_tag != 0 && rh <= E) {
+        sk_find_two(h1, SK_RBINS, k, rh, K.red, &K.fr, &K.fr2);
+        if (K.fr2.ok) hb = K.fr2.bin;
+    } else {
+        block_find_bin(h1, SK_RBINS, k, K.red, &K.fr);
     }
-    block_find_bin(h1, SK_RBINS, k, K.red, &K.fr);
     const bool ok1 = K.fr.ok;
     const uint32_t b1 = K.fr.bin;
     const uint32_t rem = k - K.fr.above;
@@ -445,11 +494,9 @@ __device__ __forceinline__ bool sk_threshold_select(const SmallParams& p, SmallS
     const uint32_t s2 = sh > 12u ? sh - 12u : 0u;          // bits left for pass 3
     const uint32_t nb2 = max(1u << (sh - s2), 512u);
     const uint32_t lmask = (1u << sh) - 1u;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint32_t q = (uint32_t)tid + (uint32_t)u * SK_THREADS;
-        const uint32_t r = key[u] - T0;
-        if (q < E && (r >> sh) == b1) atomicAdd(&h2[(r & lmask) >> s2], 1u);
+    for (uint32_t q = tid; q < E; q += SK_THREADS) {
+        const uint32_t r = K.ckey[q] - T0;
+        if ((r >> sh) == b1) atomicAdd(&h2[(r & lmask) >> s2], 1u);
     }
     __syncthreads();
     mark_phase(p.ctrl, 5);
@@ -464,11 +511,9 @@ __device__ __forceinline__ bool sk_threshold_select(const SmallParams& p, SmallS
         for (int i = tid; i < 512; i += SK_THREADS) h1[i] = 0;
         __syncthreads();
         const uint32_t pre3 = (b1 << (sh - s2)) | t2;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t q = (uint32_t)tid + (uint32_t)u * SK_THREADS;
-            const uint32_t r = key[u] - T0;
-            if (q < E && (r >> s2) == pre3) atomicAdd(&h1[r & ((1u << s2) - 1u)], 1u);
+        for (uint32_t q = tid; q < E; q += SK_THREADS) {
+            const uint32_t r = K.ckey[q] - T0;
+            if ((r >> s2) == pre3) atomicAdd(&h1[r & ((1u << s2) - 1u)], 1u);
         }
         __syncthreads();
         block_find_bin(h1, 512, rem2, K.red, &K.fr);
@@ -482,13 +527,10 @@ __device__ __forceinline__ bool sk_threshold_select(const SmallParams& p, SmallS
     // shared-memory add per warp
     const uint32_t before = K.pre_blk[c];
     uint32_t g = 0, e = 0;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint32_t q = (uint32_t)tid + (uint32_t)u * SK_THREADS;
-        if (q < before) {
-            g += key[u] > Tk;
-            e += key[u] == Tk;
-        }
+    for (uint32_t q = tid; q < before; q += SK_THREADS) {
+        const uint32_t key = K.ckey[q];
+        g += key > Tk;
+        e += key == Tk;
     }
     g = __reduce_add_sync(~0u, g);
     e = __reduce_add_sync(~0u, e);
@@ -643,7 +685,7 @@ small_kernel(const __grid_constant__ SmallParams p) {
             [&](uint32_t i, uint32_t j) {
                 p.cand_idx[e0 + j] = (uint32_t)(e0 + i);
                 p.cand_val[e0 + j] = K.acc[i];
-                K.own[j] = i;
+                if (j < SK_CAP1) K.own[j] = i;
             });
     }
     mark_phase(ctrl, 1);
@@ -859,7 +901,6 @@ small_kernel(const __grid_constant__ SmallParams p) {
             before_eq = s_out[3];
         }
     }
-    mark_phase(ctrl, 6);
 
     // ---- 5: emission in index order from shared memory: the threshold path
     // only looks at the block's own candidates (one warp), the exact path at
