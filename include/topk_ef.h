@@ -35,7 +35,9 @@
  *    (device memory, at least the size the matching *_workspace_bytes call
  *    returns, 256-byte aligned).  Calls on the same workspace must be ordered
  *    (same stream, or synchronised); the library allocates no memory and
- *    keeps nothing between calls except inside `ws`.
+ *    keeps nothing between calls except inside `ws`.  A workspace needs no
+ *    initialisation: its contents before the first call (zeros, garbage, a
+ *    workspace last used with other sizes) never change a result.
  *  - fp32 arrays must be 4-byte aligned; 16-byte aligned grad/residual take
  *    the vectorised path, other alignments a scalar path with identical
  *    results.
@@ -89,6 +91,17 @@ size_t topk_ef_workspace_bytes(int64_t n, int64_t k);
  *   out_idx   device, int32[k], ascending indices of the sent entries
  *   out_val   device, fp32[k], acc at those indices (signed)
  *   ws        device workspace of ws_bytes >= topk_ef_workspace_bytes(n, k)
+ *
+ * The compress keeps, in `ws`, the threshold of the previous call made with
+ * the same residual pointer, n, k and lr ("Sparsified SGD with Memory",
+ * abstract: the memory carries over from step to step, and so does the
+ * magnitude of what is sent): a prefilter only, the result is exact whatever
+ * it holds.  A tensor small enough for one wave of blocks (n <= 148 * 16,384
+ * on a 148-SM device) takes one kernel launch; its workspace holds 8 n bytes
+ * of candidate lists besides.  The launch's parameters are the same from
+ * call to call apart from a host-issued call number, and the kernel keeps
+ * its own call counter in `ws`, so a call captured in a CUDA graph may be
+ * replayed.
  */
 int topk_ef_compress(const float* grad, float* residual, int64_t n, float lr,
                      int64_t k, int32_t* out_idx, float* out_val, void* ws,
@@ -295,6 +308,8 @@ const char* topk_ef_status_string(int status);
 /*
  * Diagnostics of the last compress call on `ws` (synchronises `stream`):
  *   info[0]  path taken: 0 = candidate prefilter, 1 = full rescan fallback
+ *            (a small tensor: 1 = the previous call's threshold did not
+ *            decide the top k, so every block ran the exact select)
  *   info[1]  candidates kept by the prefilter
  *   info[2]  candidate capacity of the workspace
  *   info[3]  kernels launched by that call
