@@ -77,6 +77,7 @@ struct McFixed {
     uint32_t live_tot;
     uint32_t E, pre_above;
     FindResult fr;
+    uint32_t sel[8];                                  // the gathered select's results (local)
 };
 
 template <int CL>
@@ -108,20 +109,32 @@ __device__ __forceinline__ void cluster_find(cg::cluster_group& cl, McFixed& S, 
     block_find_bin(S.tot, NB, rem, S.red, &S.fr);
 }
 
-// Local histogram of `nb` bins over the gathered list (entries whose `sel`
-// holds), then the bin of the rem-th largest (result in S.fr).
-template <class Sel, class Bin>
-__device__ __forceinline__ void list_find(McFixed& S, const uint32_t* list, uint32_t E, int nb,
-                                          uint32_t rem, Sel sel, Bin bin) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) S.tot[i] = 0;
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < E; i += blockDim.x) {
-        const uint32_t v = list[i];
-        if (sel(v)) atomicAdd(&S.tot[bin(v)], 1u);
-    }
-    __syncthreads();
-    block_find_bin(S.tot, nb, rem, S.red, &S.fr);
+// One warp: the bin of the rem-th largest in a 1024-bin shared-memory
+// histogram.  Lane l sums bins [1024 - 32 (l + 1), 1024 - 32 l) (rotated so
+// that no two lanes hit one bank); a scan finds the lane whose bins hold it,
+// and a second scan over that lane's bins, one per lane, the bin.  Every
+// lane gets the result; false when the histogram holds fewer than rem.
+__device__ __forceinline__ bool warp_find_1024(const uint32_t* h, uint32_t rem, uint32_t& bin,
+                                               uint32_t& above) {
+    const uint32_t lane = lane_id();
+    const int hi = 1024 - 32 * (int)lane, lo = hi - 32;
+    uint32_t s = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) s += h[lo + ((j + (int)lane) & 31)];
+    const uint32_t incl = warp_incl_scan(s);
+    const uint32_t who = __ballot_sync(0xFFFFFFFFu, incl - s < rem && incl >= rem);
+    if (!who) return false;
+    const int src = __ffs(who) - 1;
+    const uint32_t ex = __shfl_sync(0xFFFFFFFFu, incl - s, src);
+    // that lane's 32 bins, one per lane from the top down
+    const int top = 1024 - 32 * src - 1;
+    const uint32_t c = h[top - (int)lane];
+    const uint32_t inc2 = ex + warp_incl_scan(c);
+    const uint32_t who2 = __ballot_sync(0xFFFFFFFFu, inc2 - c < rem && inc2 >= rem);
+    const int src2 = __ffs(who2) - 1;
+    bin = (uint32_t)(top - src2);
+    above = __shfl_sync(0xFFFFFFFFu, inc2 - c, src2);
+    return true;
 }
 
 template <int CL>
@@ -387,33 +400,71 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             if (i + 3 >= nr) v.w = SENT;
             g4[u] = v;
         }
+        __syncthreads();
         if (kp > 0 && ok) {
-            // bits 19..10, then 9..0 of the k-th key inside bin b1
-            list_find(S, glist, E, 1024, rem, [](uint32_t v) { return v != 0xFFFFFFFFu; },
-                      [](uint32_t v) { return (v >> 10) & 1023u; });
-            const uint32_t bA = S.fr.bin;
-            const uint32_t remA = rem - S.fr.above;
-            ok = S.fr.ok;
-            list_find(S, glist, E, 1024, remA,
-                      [bA](uint32_t v) { return v != 0xFFFFFFFFu && ((v >> 10) & 1023u) == bA; },
-                      [](uint32_t v) { return v & 1023u; });
-            ok = ok && S.fr.ok;
-            const uint32_t t = (bA << 10) | S.fr.bin;
-            q = remA - S.fr.above;
-            T = ok ? (b1 << 20) | t : NO_KEY;
-            // entries of earlier CTAs in bin b1: above T, equal to T
-            uint32_t g = 0, e = 0;
+            // bits 19..10, then 9..0 of the k-th key inside bin b1: every
+            // thread counts its share of the list into the (zeroed, here
+            // unused) digit-2 and -3 histograms, warp 0 alone finds the bins
+            // (a block-wide find costs four barriers, the warp's none)
+            constexpr uint32_t SENT_ = 0xFFFFFFFFu;
             for (uint32_t i = tid; i < E; i += blockDim.x) {
                 const uint32_t v = glist[i];
-                if ((int)(v >> 20) < cr) {
-                    g += (v & 0xFFFFFu) > t;
-                    e += (v & 0xFFFFFu) == t;
+                if (v != SENT_) atomicAdd(&S.h2[(v >> 10) & 1023u], 1u);
+            }
+            if (tid == 0) S.sel[6] = S.sel[7] = 0;
+            __syncthreads();
+            if (tid < 32) {
+                uint32_t bA = 0, aA = 0;
+                const bool f = warp_find_1024(S.h2, rem, bA, aA);
+                if (tid == 0) {
+                    S.sel[0] = f ? 1u : 0u;
+                    S.sel[1] = bA;
+                    S.sel[2] = aA;
                 }
             }
-            g = block_sum(g, S.red);
-            e = block_sum(e, S.red);
-            pg = pre_above + g;
-            pe = e;
+            __syncthreads();
+            const uint32_t bA = S.sel[1];
+            const uint32_t remA = rem - S.sel[2];
+            ok = S.sel[0] != 0;
+            if (ok) {
+                for (uint32_t i = tid; i < E; i += blockDim.x) {
+                    const uint32_t v = glist[i];
+                    if (v != SENT_ && ((v >> 10) & 1023u) == bA) atomicAdd(&S.h3[v & 1023u], 1u);
+                }
+                __syncthreads();
+                if (tid < 32) {
+                    uint32_t bB = 0, aB = 0;
+                    const bool f = warp_find_1024(S.h3, remA, bB, aB);
+                    if (tid == 0) {
+                        S.sel[3] = f ? 1u : 0u;
+                        S.sel[4] = bB;
+                        S.sel[5] = aB;
+                    }
+                }
+                __syncthreads();
+                ok = S.sel[3] != 0;
+                const uint32_t t = (bA << 10) | S.sel[4];
+                q = remA - S.sel[5];
+                T = ok ? (b1 << 20) | t : NO_KEY;
+                // entries of earlier CTAs in bin b1: above T, equal to T
+                uint32_t g = 0, e = 0;
+                for (uint32_t i = tid; i < E; i += blockDim.x) {
+                    const uint32_t v = glist[i];
+                    if (v != SENT_ && (int)(v >> 20) < cr) {
+                        g += (v & 0xFFFFFu) > t;
+                        e += (v & 0xFFFFFu) == t;
+                    }
+                }
+                g = __reduce_add_sync(0xFFFFFFFFu, g);
+                e = __reduce_add_sync(0xFFFFFFFFu, e);
+                if (lane_id() == 0 && (g | e)) {
+                    atomicAdd(&S.sel[6], g);
+                    atomicAdd(&S.sel[7], e);
+                }
+                __syncthreads();
+                pg = pre_above + S.sel[6];
+                pe = S.sel[7];
+            }
         }
     } else {
         // crowded bin: two more summed digit passes, then exact counts
