@@ -49,14 +49,38 @@ merge_setup_kernel(const MergeSetupParams p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((uint32_t)b < p.validate_blocks) {
+        // a contiguous range of the P * k_in entries per block; each thread's
+        // position inside its row is carried along (no division per entry),
+        // and four entries and their successors are loaded at once
         const int64_t tot = (int64_t)p.P * p.k_in;
+        const int64_t per = (tot + p.validate_blocks - 1) / p.validate_blocks;
+        const int64_t e0 = min((int64_t)b * per, tot), e1 = min(e0 + per, tot);
         bool bad = false;
-        for (int64_t e = (int64_t)b * blockDim.x + tid; e < tot;
-             e += (int64_t)p.validate_blocks * blockDim.x) {
-            const int64_t j = e % p.k_in;
-            const int32_t v = p.in_idx[e];
-            if (v < 0 || (int64_t)v >= p.n) bad = true;
-            if (j + 1 < p.k_in && p.in_idx[e + 1] <= v) bad = true;
+        int64_t e = e0 + tid;
+        int64_t j = e % p.k_in;                  // position of entry e in its row
+        const int64_t step = (int64_t)blockDim.x;
+        const int64_t jstep = step % p.k_in;
+        while (e < e1) {
+            int32_t v[4], w[4];
+            bool last[4];
+            int64_t ee = e, jj = j;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                last[u] = jj + 1 >= p.k_in;      // no successor in the row
+                v[u] = ee < e1 ? p.in_idx[ee] : 0;
+                w[u] = (ee < e1 && !last[u]) ? p.in_idx[ee + 1] : 0;
+                ee += step;
+                jj += jstep;
+                if (jj >= p.k_in) jj -= p.k_in;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (e + u * step >= e1) break;
+                if (v[u] < 0 || (int64_t)v[u] >= p.n) bad = true;
+                if (!last[u] && w[u] <= v[u]) bad = true;
+            }
+            e = ee;
+            j = jj;
         }
         const int any = __syncthreads_or(bad);
         if (tid == 0) p.bad_words[b] = any ? 1u : 0u;

@@ -109,32 +109,41 @@ __device__ __forceinline__ void cluster_find(cg::cluster_group& cl, McFixed& S, 
     block_find_bin(S.tot, NB, rem, S.red, &S.fr);
 }
 
-// One warp: the bin of the rem-th largest in a 1024-bin shared-memory
-// histogram.  Lane l sums bins [1024 - 32 (l + 1), 1024 - 32 l) (rotated so
-// that no two lanes hit one bank); a scan finds the lane whose bins hold it,
-// and a second scan over that lane's bins, one per lane, the bin.  Every
-// lane gets the result; false when the histogram holds fewer than rem.
-__device__ __forceinline__ bool warp_find_1024(const uint32_t* h, uint32_t rem, uint32_t& bin,
-                                               uint32_t& above) {
+// One warp: the bin of the rem-th largest in an NB-bin shared-memory
+// histogram (NB a multiple of 1024).  Lane l sums the W = NB / 32 bins
+// [NB - W (l + 1), NB - W l) (rotated so that no two lanes hit one bank); a
+// scan finds the lane whose bins hold it, then scans over that lane's bins,
+// 32 at a time from the top, the bin.  Every lane gets the result; false
+// when the histogram holds fewer than rem.  No block barrier.
+template <int NB>
+__device__ __forceinline__ bool warp_find(const uint32_t* h, uint32_t rem, uint32_t& bin,
+                                          uint32_t& above) {
+    constexpr int W = NB / 32;
+    static_assert(W % 32 == 0, "whole bank rows per lane");
     const uint32_t lane = lane_id();
-    const int hi = 1024 - 32 * (int)lane, lo = hi - 32;
+    const int lo = NB - W * ((int)lane + 1);
     uint32_t s = 0;
 #pragma unroll 8
-    for (int j = 0; j < 32; ++j) s += h[lo + ((j + (int)lane) & 31)];
+    for (int j = 0; j < W; ++j) s += h[lo + ((j + (int)lane) & (W - 1))];
     const uint32_t incl = warp_incl_scan(s);
     const uint32_t who = __ballot_sync(0xFFFFFFFFu, incl - s < rem && incl >= rem);
     if (!who) return false;
     const int src = __ffs(who) - 1;
-    const uint32_t ex = __shfl_sync(0xFFFFFFFFu, incl - s, src);
-    // that lane's 32 bins, one per lane from the top down
-    const int top = 1024 - 32 * src - 1;
-    const uint32_t c = h[top - (int)lane];
-    const uint32_t inc2 = ex + warp_incl_scan(c);
-    const uint32_t who2 = __ballot_sync(0xFFFFFFFFu, inc2 - c < rem && inc2 >= rem);
-    const int src2 = __ffs(who2) - 1;
-    bin = (uint32_t)(top - src2);
-    above = __shfl_sync(0xFFFFFFFFu, inc2 - c, src2);
-    return true;
+    uint32_t run = __shfl_sync(0xFFFFFFFFu, incl - s, src);
+    const int top = NB - W * src - 1;
+    for (int c0 = 0; c0 < W; c0 += 32) {
+        const uint32_t cnt = h[top - c0 - (int)lane];
+        const uint32_t inc2 = run + warp_incl_scan(cnt);
+        const uint32_t who2 = __ballot_sync(0xFFFFFFFFu, inc2 - cnt < rem && inc2 >= rem);
+        if (who2) {
+            const int src2 = __ffs(who2) - 1;
+            bin = (uint32_t)(top - c0 - src2);
+            above = __shfl_sync(0xFFFFFFFFu, inc2 - cnt, src2);
+            return true;
+        }
+        run = __shfl_sync(0xFFFFFFFFu, inc2, 31);
+    }
+    return false;
 }
 
 template <int CL>
@@ -319,7 +328,16 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             reinterpret_cast<uint4*>(S.tot)[t] = v;
         }
         __syncthreads();
-        block_find_bin(S.tot, D1_BINS, rem, S.red, &S.fr);
+        if (tid < 32) {
+            uint32_t bb = 0, ab = 0;
+            const bool f = warp_find<D1_BINS>(S.tot, rem, bb, ab);
+            if (tid == 0) {
+                S.fr.ok = f ? 1u : 0u;
+                S.fr.bin = bb;
+                S.fr.above = ab;
+            }
+        }
+        __syncthreads();
         ok = S.fr.ok;
         b1 = S.fr.bin;
         rem -= S.fr.above;
@@ -415,7 +433,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             __syncthreads();
             if (tid < 32) {
                 uint32_t bA = 0, aA = 0;
-                const bool f = warp_find_1024(S.h2, rem, bA, aA);
+                const bool f = warp_find<D2_BINS>(S.h2, rem, bA, aA);
                 if (tid == 0) {
                     S.sel[0] = f ? 1u : 0u;
                     S.sel[1] = bA;
@@ -434,7 +452,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
                 __syncthreads();
                 if (tid < 32) {
                     uint32_t bB = 0, aB = 0;
-                    const bool f = warp_find_1024(S.h3, remA, bB, aB);
+                    const bool f = warp_find<D3_BINS>(S.h3, remA, bB, aB);
                     if (tid == 0) {
                         S.sel[3] = f ? 1u : 0u;
                         S.sel[4] = bB;
