@@ -29,6 +29,7 @@ struct MergeSetupParams {
     uint64_t zero_vec4;
     uint32_t* bad_words;    // [validate_blocks], one verdict per block
     uint32_t* sizes;        // [P]
+    uint32_t* floors;       // [P] lower key bound of each set (0: none known)
     uint32_t* set_idx;      // [P][set_cap]
     float* set_val;
     int64_t set_cap;
@@ -95,7 +96,10 @@ merge_setup_kernel(const MergeSetupParams p) {
             c.kernels = p.kernels;
             *p.ctrl = c;
         }
-        for (int i = tid; i < p.P; i += blockDim.x) p.sizes[i] = (uint32_t)p.k_in;
+        for (int i = tid; i < p.P; i += blockDim.x) {
+            p.sizes[i] = (uint32_t)p.k_in;
+            p.floors[i] = 0;
+        }
         if (p.lonely >= 0) {
             const int64_t src = (int64_t)p.lonely * p.k_in;
             const int64_t dst = (int64_t)p.lonely * p.set_cap;

@@ -41,6 +41,22 @@ struct McCfg {
     static constexpr int GCAP = STAGE - QMAX - 4;                     // gathered list capacity
 };
 
+// Relative digit 1 (rounds after the first): bin 0 holds the keys below the
+// pair's floor L (sums at common indices can fall there), bins 1 .. 2046 the
+// keys in [L + (b - 1) 2^13, L + b 2^13) (two octaves above L), bin 2047 the
+// rest; the k-th key in bin 0 or 2047, or a bin too crowded to gather,
+// repeats the digit with key >> 20.
+constexpr int MC_RSH = 13;
+
+__device__ __forceinline__ uint32_t mc_bin(uint32_t key, bool rel, uint32_t L) {
+    if (!rel) return key >> 20;
+    if (key < L) return 0u;
+    return min(((key - L) >> MC_RSH) + 1u, (uint32_t)(D1_BINS - 1));
+}
+__device__ __forceinline__ uint32_t mc_low(uint32_t key, bool rel, uint32_t L) {
+    return rel ? ((key - L) & ((1u << MC_RSH) - 1u)) : (key & 0xFFFFFu);
+}
+
 struct MergeClusterParams {
     const uint32_t* src_idx;     // sets of this round, row stride src_stride
     const float* src_val;
@@ -53,6 +69,9 @@ struct MergeClusterParams {
     float* dst_val;
     int64_t dst_stride;
     uint32_t* sizes_out;
+    const uint32_t* floor_in;    // null (first round): digit 1 is key >> 20; else each set's
+                                 // lowest key, and digit 1 is relative to the pair's lower one
+    uint32_t* floor_out;         // the merged set's lowest key (its k-th)
     int32_t final_out;           // last round: the caller's arrays
     int32_t* out_idx;
     float* out_val;
@@ -176,6 +195,13 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     }
     const int64_t left = (int64_t)pair * 2 * p.step;
     const int64_t right = left + p.step;
+    // digit 1 relative to the pair's lower floor when both are known
+    uint32_t Lf = 0;
+    bool rel = false;
+    if (p.floor_in) {
+        Lf = min(p.floor_in[left], p.floor_in[right]);
+        rel = Lf != 0;
+    }
     int64_t a = p.sizes_in ? p.sizes_in[left] : p.size_const;
     int64_t b = p.sizes_in ? p.sizes_in[right] : p.size_const;
     a = a < p.src_stride ? a : p.src_stride;
@@ -287,13 +313,31 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             mv[u] = oi == DEAD ? 0.f : ov;
             if (oi != DEAD) {
                 ++live;
-                atomicAdd(&S.h1[key_of(mv[u]) >> 20], 1u);
+                atomicAdd(&S.h1[mc_bin(key_of(mv[u]), rel, Lf)], 1u);
             }
         }
     }
     live = block_sum(live, S.red);
     if (tid == 0) S.live = live;
     if (stamp) p.ctrl->t_phase[3] = global_ns();
+    uint32_t kp = 0, b1 = 0, rem = 0;
+    bool ok = false;
+    uint32_t* mylist = stage;                           // [QMAX]
+    uint32_t* glist = stage + QMAX + 4;                 // [GCAP]
+    constexpr uint32_t SENT = 0xFFFFFFFFu;              // padding entry of the lists
+    for (int attempt = 0;; ++attempt) {
+    if (attempt > 0) {
+        // the relative digit did not decide: every CTA is past its reads of
+        // the others' slices and lists; digit 1 again with key >> 20
+        rel = false;
+        cl.sync();
+        for (int i = tid; i < D1_BINS; i += blockDim.x) S.h1[i] = 0;
+        for (int i = tid; i < D1_BINS / CL; i += blockDim.x) S.hslice[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < PT; ++u)
+            if (mi[u] != DEAD) atomicAdd(&S.h1[key_of(mv[u]) >> 20], 1u);
+    }
     cl.sync();                                           // [1] h1 and live of every CTA
     if (stamp) p.ctrl->t_phase[4] = global_ns();
 
@@ -316,9 +360,10 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     }
     cl.sync();                                           // [1b] every slice summed
     const uint32_t live_tot = S.live_tot;
-    const uint32_t kp = live_tot < p.kmax ? live_tot : p.kmax;
-    uint32_t b1 = 0, rem = kp;
-    bool ok = kp > 0;
+    kp = live_tot < p.kmax ? live_tot : p.kmax;
+    b1 = 0;
+    rem = kp;
+    ok = kp > 0;
     if (kp > 0) {
         // the summed histogram from its CL owners, 16 bytes per thread
         for (int t = tid; t < D1_BINS / 4; t += blockDim.x) {
@@ -344,14 +389,12 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     }
     // this CTA's entries in bin b1 (low 20 key bits, in the staging space,
     // which the merge no longer needs) and its count above b1
-    uint32_t* mylist = stage;                           // [QMAX]
-    uint32_t* glist = stage + QMAX + 4;                 // [GCAP]
     {
         uint32_t nin = 0, nab = 0;
 #pragma unroll
         for (int u = 0; u < PT; ++u) {
             if (mi[u] == DEAD || kp == 0) continue;
-            const uint32_t d = key_of(mv[u]) >> 20;
+            const uint32_t d = mc_bin(key_of(mv[u]), rel, Lf);
             nin += d == b1;
             nab += d > b1;
         }
@@ -362,7 +405,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         for (int u = 0; u < PT; ++u) {
             if (mi[u] == DEAD || kp == 0) continue;
             const uint32_t key = key_of(mv[u]);
-            if ((key >> 20) == b1) mylist[at++] = ((uint32_t)cr << 20) | (key & 0xFFFFFu);
+            if (mc_bin(key, rel, Lf) == b1) mylist[at++] = ((uint32_t)cr << 20) | mc_low(key, rel, Lf);
         }
         nab = block_sum(nab, S.red);
         if (tid == 0) {
@@ -375,7 +418,6 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
 
     // list lengths and counts above b1 of all CTAs (lane r reads rank r);
     // in the gathered list each CTA's entries start at a multiple of 4
-    constexpr uint32_t SENT = 0xFFFFFFFFu;              // padding entry
     if (tid < 32) {
         const uint32_t lane = lane_id();
         uint32_t nr = 0, ar = 0;
@@ -398,6 +440,12 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         }
     }
     __syncthreads();
+    // the relative digit decides unless the k-th key is in an open bin or
+    // its bin is too crowded to gather (the same in every CTA)
+    if (!rel || kp == 0 || (ok && b1 != 0 && b1 != (uint32_t)(D1_BINS - 1) &&
+                            S.E <= (uint32_t)C::GCAP))
+        break;
+    }
     const uint32_t E = S.E, pre_above = S.pre_above;
     uint32_t T = NO_KEY, q = 0, pg = 0, pe = 0;
     const bool gathered = E <= (uint32_t)C::GCAP;       // the same in every CTA
@@ -425,9 +473,10 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             // unused) digit-2 and -3 histograms, warp 0 alone finds the bins
             // (a block-wide find costs four barriers, the warp's none)
             constexpr uint32_t SENT_ = 0xFFFFFFFFu;
+            const uint32_t lsh = rel ? (uint32_t)MC_RSH - 10u : 10u;   // bits below pass A
             for (uint32_t i = tid; i < E; i += blockDim.x) {
                 const uint32_t v = glist[i];
-                if (v != SENT_) atomicAdd(&S.h2[(v >> 10) & 1023u], 1u);
+                if (v != SENT_) atomicAdd(&S.h2[((v & 0xFFFFFu) >> lsh) & 1023u], 1u);
             }
             if (tid == 0) S.sel[6] = S.sel[7] = 0;
             __syncthreads();
@@ -447,7 +496,8 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
             if (ok) {
                 for (uint32_t i = tid; i < E; i += blockDim.x) {
                     const uint32_t v = glist[i];
-                    if (v != SENT_ && ((v >> 10) & 1023u) == bA) atomicAdd(&S.h3[v & 1023u], 1u);
+                    if (v != SENT_ && (((v & 0xFFFFFu) >> lsh) & 1023u) == bA)
+                        atomicAdd(&S.h3[v & ((1u << lsh) - 1u)], 1u);
                 }
                 __syncthreads();
                 if (tid < 32) {
@@ -461,9 +511,9 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
                 }
                 __syncthreads();
                 ok = S.sel[3] != 0;
-                const uint32_t t = (bA << 10) | S.sel[4];
+                const uint32_t t = (bA << lsh) | S.sel[4];
                 q = remA - S.sel[5];
-                T = ok ? (b1 << 20) | t : NO_KEY;
+                T = !ok ? NO_KEY : rel ? Lf + ((b1 - 1u) << MC_RSH) + t : (b1 << 20) | t;
                 // entries of earlier CTAs in bin b1: above T, equal to T
                 uint32_t g = 0, e = 0;
                 for (uint32_t i = tid; i < E; i += blockDim.x) {
@@ -583,6 +633,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         }
     } else if (cr == 0 && tid == 0) {
         p.sizes_out[left] = kp;
+        if (p.floor_out) p.floor_out[left] = T == NO_KEY ? 0u : T;
     }
     if (stamp) p.ctrl->t_phase[7] = global_ns();
     // this CTA's shared memory stays valid until every CTA has read it

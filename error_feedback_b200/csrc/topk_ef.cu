@@ -769,7 +769,7 @@ int static_scratch_addr(void** out) {
 // --------------------------------------------------------- merge planning
 
 struct MLayout {
-    size_t ctrl, sizes, bad, zero_begin, hist, live, zero_end, slots, set_idx, set_val, m_idx,
+    size_t ctrl, sizes, floors, bad, zero_begin, hist, live, zero_end, slots, set_idx, set_val, m_idx,
         m_val, total;
     int64_t cap;
     int rounds;
@@ -806,6 +806,8 @@ MLayout merge_layout(int32_t P, int64_t k_in, int64_t k) {
     L.ctrl = o;
     o = align_up(o + sizeof(Ctrl));
     L.sizes = o;
+    o = align_up(o + (size_t)P * sizeof(uint32_t));
+    L.floors = o;
     o = align_up(o + (size_t)P * sizeof(uint32_t));
     L.bad = o;
     o = align_up(o + 148 * sizeof(uint32_t));
@@ -1068,6 +1070,7 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     char* w = (char*)ws;
     Ctrl* ctrl = reinterpret_cast<Ctrl*>(w + L.ctrl);
     uint32_t* sizes = reinterpret_cast<uint32_t*>(w + L.sizes);
+    uint32_t* floors = reinterpret_cast<uint32_t*>(w + L.floors);
     uint32_t* bad = reinterpret_cast<uint32_t*>(w + L.bad);
     uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.hist);
     uint32_t* live = reinterpret_cast<uint32_t*>(w + L.live);
@@ -1101,6 +1104,7 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     sp.zero_vec4 = cluster_path ? 0 : (L.zero_end - L.zero_begin) / 16;
     sp.bad_words = bad;
     sp.sizes = sizes;
+    sp.floors = floors;
     sp.set_idx = set_idx;
     sp.set_val = set_val;
     sp.set_cap = L.cap;
@@ -1169,6 +1173,10 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
             cp.dst_val = set_val;
             cp.dst_stride = L.cap;
             cp.sizes_out = sizes;
+            // after round 0 every set's lower key bound is known: the
+            // round's digit 1 can be relative to it
+            cp.floor_in = r == 0 ? nullptr : floors;
+            cp.floor_out = floors;
             cp.final_out = (r == L.rounds - 1) ? 1 : 0;
             cp.out_idx = out_idx;
             cp.out_val = out_val;

@@ -178,3 +178,25 @@ def test_merge_paths(P, k_in, k, n, cluster):
     rounds = (P - 1).bit_length()
     kernels = ef.topk_ef_path_info(ws)["kernels"]
     assert kernels == (1 + rounds if cluster else 1 + 2 * rounds), kernels
+
+
+@pytest.mark.parametrize("case", ["cancel", "grow"])
+def test_merge_relative_digit_falls_back(case):
+    """After the first round the cluster kernel bins digit 1 relative to the
+    lower of the two sets' lowest keys, two octaves wide; a k-th key below
+    it (values that cancel at common indices) or above it (values that add
+    up to more than four times it) repeats the digit over the whole key.
+    P = 4: round 0 builds two sets on the same indices, round 1 merges them."""
+    rng = np.random.default_rng(41)
+    n, k = 10_000, 1000
+    I = np.sort(rng.choice(n, k, replace=False))
+    J = np.sort(np.setdiff1d(rng.choice(n, 3 * k, replace=False), I)[:k])
+    x = rng.uniform(1.0, 1.1, k).astype(np.float32)
+    y = rng.uniform(0.5, 0.6, k).astype(np.float32)
+    if case == "cancel":
+        vals = [x, y, -x, -y]
+    else:
+        vals = [x, y, (np.float32(7.0) * x).astype(np.float32), y]
+    idx = np.stack([I, J, I, J]).astype(np.int32)
+    val = np.stack(vals).astype(np.float32)
+    run_merge(idx, val, k, n, ws=_mws(4, k, k))
