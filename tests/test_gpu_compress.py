@@ -450,3 +450,22 @@ def test_index_width_boundary():
     want = g.mul_(LR)
     want[gi.long()] = 0.0
     assert torch.equal(want.view(torch.int32), res.view(torch.int32))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_small_random_sequences(seed):
+    """Random small tensors (one wave of blocks, so small_kernel) with k
+    small enough for the threshold hint, eight EF steps each over gradients
+    whose scale drifts, some steps from a zeroed memory: both paths and their
+    switches, every step compared bit for bit."""
+    rng = np.random.default_rng(1000 + seed)
+    n = int(rng.integers(1, 2_400_000))
+    k = int(rng.integers(1, min(n, 2048) + 1))
+    offset = int(rng.integers(0, 4))
+    scales = np.exp(rng.normal(0.0, 0.3, 8)).astype(np.float32)
+    grads = [(rng.standard_normal(n) * s).astype(np.float32) for s in scales]
+    ws = _ws(n, k)
+    paths = []
+    run_compress_steps(grads, LR, k, offset_elems=offset, ws=ws, paths=paths,
+                       zero_between=bool(seed % 2))
+    assert all(p["kernels"] == 1 for p in paths), paths
