@@ -294,6 +294,43 @@ __device__ __forceinline__ void block_find_bin(const uint32_t* h, int nb, uint32
     __syncthreads();
 }
 
+// One warp: the bin of the rem-th largest in an NB-bin shared-memory
+// histogram (NB a multiple of 1024).  Lane l sums the W = NB / 32 bins
+// [NB - W (l + 1), NB - W l) (rotated so that no two lanes hit one bank); a
+// scan finds the lane whose bins hold it, then scans over that lane's bins,
+// 32 at a time from the top, the bin.  Every lane gets the result; false
+// when the histogram holds fewer than rem.  No block barrier.
+template <int NB>
+__device__ __forceinline__ bool warp_find(const uint32_t* h, uint32_t rem, uint32_t& bin,
+                                          uint32_t& above) {
+    constexpr int W = NB / 32;
+    static_assert(W % 32 == 0, "whole bank rows per lane");
+    const uint32_t lane = lane_id();
+    const int lo = NB - W * ((int)lane + 1);
+    uint32_t s = 0;
+#pragma unroll 8
+    for (int j = 0; j < W; ++j) s += h[lo + ((j + (int)lane) & (W - 1))];
+    const uint32_t incl = warp_incl_scan(s);
+    const uint32_t who = __ballot_sync(0xFFFFFFFFu, incl - s < rem && incl >= rem);
+    if (!who) return false;
+    const int src = __ffs(who) - 1;
+    uint32_t run = __shfl_sync(0xFFFFFFFFu, incl - s, src);
+    const int top = NB - W * src - 1;
+    for (int c0 = 0; c0 < W; c0 += 32) {
+        const uint32_t cnt = h[top - c0 - (int)lane];
+        const uint32_t inc2 = run + warp_incl_scan(cnt);
+        const uint32_t who2 = __ballot_sync(0xFFFFFFFFu, inc2 - cnt < rem && inc2 >= rem);
+        if (who2) {
+            const int src2 = __ffs(who2) - 1;
+            bin = (uint32_t)(top - c0 - src2);
+            above = __shfl_sync(0xFFFFFFFFu, inc2 - cnt, src2);
+            return true;
+        }
+        run = __shfl_sync(0xFFFFFFFFu, inc2, 31);
+    }
+    return false;
+}
+
 // Shared-memory histogram increment, aggregated over the lanes of a warp
 // that hit the same bin (the active lanes are given by `active`).
 __device__ __forceinline__ void warp_agg_inc(uint32_t* h, uint32_t bin, bool active) {
