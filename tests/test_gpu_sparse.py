@@ -63,8 +63,12 @@ def test_return_gtopk_p32_full():
 
 @pytest.mark.parametrize("P,k,n,kg", [(1, 10, 100, 5), (3, 1000, 50_000, 1500),
                                       (8, 4096, 1 << 20, 8192), (5, 1, 10, 0),
-                                      (2, 5000, 5000, 5000), (4, 0, 100, 10)])
+                                      (2, 5000, 5000, 5000), (4, 0, 100, 10),
+                                      (4, 50_000, 1_000_000, 40_960),
+                                      (4, 50_000, 1_000_000, 60_000)])
 def test_return_shapes(P, k, n, kg):
+    """Global lists from empty to far longer than the kernel's 4,096-entry
+    shared-memory sample (long stretches between two samples)."""
     rng = np.random.default_rng(P * 100 + k)
     idx = _sets(rng, P, k, n) if k else np.zeros((P, 0), np.int32)
     val = rng.standard_normal((P, k)).astype(np.float32)
