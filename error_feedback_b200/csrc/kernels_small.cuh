@@ -106,6 +106,8 @@ struct SmallShared {
     uint64_t tag, seq;
     uint32_t T0, sh, E, armed;
     uint32_t cnt[2];            // threshold path: earlier candidates above / at T
+    uint32_t lkey[64], lpos[64];        // threshold path: the k-th key's bin, when short
+    uint32_t lcnt, lsel[3];
 };
 
 struct SmallParams {
@@ -490,53 +492,121 @@ __device__ __forceinline__ bool sk_threshold_select(const SmallParams& p, SmallS
     const uint32_t b1 = K.fr.bin;
     const uint32_t rem = k - K.fr.above;
     if (!ok1 || b1 == (uint32_t)(SK_RBINS - 1)) return false;
-    // ---- pass 2: the bits below the bin (their top 12 when there are more)
-    const uint32_t s2 = sh > 12u ? sh - 12u : 0u;          // bits left for pass 3
-    const uint32_t nb2 = max(1u << (sh - s2), 512u);
-    const uint32_t lmask = (1u << sh) - 1u;
-    for (uint32_t q = tid; q < E; q += SK_THREADS) {
-        const uint32_t r = K.ckey[q] - T0;
-        if ((r >> sh) == b1) atomicAdd(&h2[(r & lmask) >> s2], 1u);
-    }
-    __syncthreads();
-    mark_phase(p.ctrl, 5);
-    block_find_bin(h2, (int)nb2, rem, K.red, &K.fr);
-    const bool ok2 = K.fr.ok;
-    const uint32_t t2 = K.fr.bin;
-    uint32_t rem2 = rem - K.fr.above;
-    uint32_t low = t2 << s2;
-    bool ok3 = true;
-    if (s2 > 0) {
-        // ---- pass 3 (threshold 0 only): the last s2 bits, in pass 1's words
-        for (int i = tid; i < 512; i += SK_THREADS) h1[i] = 0;
-        __syncthreads();
-        const uint32_t pre3 = (b1 << (sh - s2)) | t2;
+    const uint32_t before = K.pre_blk[c];
+    uint32_t Tk, rem2;
+    if (K.fr.cnt <= 64u) {
+        // ---- a short bin (the usual case): its entries into a list, with
+        // the earlier blocks' candidates in higher bins counted on the way;
+        // one warp then ranks the list
+        uint32_t g = 0;
         for (uint32_t q = tid; q < E; q += SK_THREADS) {
-            const uint32_t r = K.ckey[q] - T0;
-            if ((r >> s2) == pre3) atomicAdd(&h1[r & ((1u << s2) - 1u)], 1u);
+            const uint32_t key = K.ckey[q];
+            const uint32_t bin = min((key - T0) >> sh, (uint32_t)(SK_RBINS - 1));
+            if (bin == b1) {
+                const uint32_t at = atomicAdd(&K.lcnt, 1u);
+                K.lkey[at] = key;
+                K.lpos[at] = q;
+            } else if (bin > b1 && q < before) {
+                ++g;
+            }
+        }
+        g = __reduce_add_sync(~0u, g);
+        if (lane_id() == 0 && g) atomicAdd(&K.cnt[0], g);
+        __syncthreads();
+        mark_phase(p.ctrl, 5);
+        if (tid < 32) {
+            const uint32_t n1 = K.lcnt;
+            // the rem-th largest key of the list: the key with fewer than rem
+            // larger ones and at least rem at least as large
+            uint32_t Tsel = 0;
+            bool found = false;
+            for (uint32_t j = tid; j < n1; j += 32) {
+                const uint32_t kj = K.lkey[j];
+                uint32_t gt = 0, ge = 0;
+                for (uint32_t i = 0; i < n1; ++i) {
+                    const uint32_t ki = K.lkey[i];
+                    gt += ki > kj;
+                    ge += ki >= kj;
+                }
+                if (gt < rem && rem <= ge) {
+                    found = true;
+                    Tsel = kj;
+                }
+            }
+            const uint32_t who = __ballot_sync(~0u, found);
+            const uint32_t T = who ? __shfl_sync(~0u, Tsel, __ffs(who) - 1) : 0u;
+            uint32_t ga = 0, gb = 0, eb = 0;
+            for (uint32_t j = tid; j < n1; j += 32) {
+                const uint32_t kj = K.lkey[j];
+                ga += kj > T;
+                if (K.lpos[j] < before) {
+                    gb += kj > T;
+                    eb += kj == T;
+                }
+            }
+            ga = warp_sum(ga);
+            gb = warp_sum(gb);
+            eb = warp_sum(eb);
+            if (tid == 0) {
+                K.lsel[0] = who ? 1u : 0u;
+                K.lsel[1] = T;
+                K.lsel[2] = rem - ga;
+                K.cnt[0] += gb;
+                K.cnt[1] = eb;
+            }
         }
         __syncthreads();
-        block_find_bin(h1, 512, rem2, K.red, &K.fr);
-        ok3 = K.fr.ok;
-        low |= K.fr.bin;
-        rem2 -= K.fr.above;
-    }
-    if (!ok2 || !ok3) return false;
-    const uint32_t Tk = T0 + (b1 << sh) + low;
-    // ---- earlier blocks' candidates above / equal to T: per warp, then one
-    // shared-memory add per warp
-    const uint32_t before = K.pre_blk[c];
-    uint32_t g = 0, e = 0;
-    for (uint32_t q = tid; q < before; q += SK_THREADS) {
-        const uint32_t key = K.ckey[q];
-        g += key > Tk;
-        e += key == Tk;
-    }
-    g = __reduce_add_sync(~0u, g);
-    e = __reduce_add_sync(~0u, e);
-    if (lane_id() == 0 && (g | e)) {
-        atomicAdd(&K.cnt[0], g);
-        atomicAdd(&K.cnt[1], e);
+        if (!K.lsel[0]) return false;
+        Tk = K.lsel[1];
+        rem2 = K.lsel[2];
+    } else {
+        // ---- pass 2: the bits below the bin (their top 12 when there are more)
+        const uint32_t s2 = sh > 12u ? sh - 12u : 0u;          // bits left for pass 3
+        const uint32_t nb2 = max(1u << (sh - s2), 512u);
+        const uint32_t lmask = (1u << sh) - 1u;
+        for (uint32_t q = tid; q < E; q += SK_THREADS) {
+            const uint32_t r = K.ckey[q] - T0;
+            if ((r >> sh) == b1) atomicAdd(&h2[(r & lmask) >> s2], 1u);
+        }
+        __syncthreads();
+        mark_phase(p.ctrl, 5);
+        block_find_bin(h2, (int)nb2, rem, K.red, &K.fr);
+        const bool ok2 = K.fr.ok;
+        const uint32_t t2 = K.fr.bin;
+        rem2 = rem - K.fr.above;
+        uint32_t low = t2 << s2;
+        bool ok3 = true;
+        if (s2 > 0) {
+            // ---- pass 3 (threshold 0 only): the last s2 bits, in pass 1's words
+            for (int i = tid; i < 512; i += SK_THREADS) h1[i] = 0;
+            __syncthreads();
+            const uint32_t pre3 = (b1 << (sh - s2)) | t2;
+            for (uint32_t q = tid; q < E; q += SK_THREADS) {
+                const uint32_t r = K.ckey[q] - T0;
+                if ((r >> s2) == pre3) atomicAdd(&h1[r & ((1u << s2) - 1u)], 1u);
+            }
+            __syncthreads();
+            block_find_bin(h1, 512, rem2, K.red, &K.fr);
+            ok3 = K.fr.ok;
+            low |= K.fr.bin;
+            rem2 -= K.fr.above;
+        }
+        if (!ok2 || !ok3) return false;
+        Tk = T0 + (b1 << sh) + low;
+        // ---- earlier blocks' candidates above / equal to T: per warp, then
+        // one shared-memory add per warp
+        uint32_t g = 0, e = 0;
+        for (uint32_t q = tid; q < before; q += SK_THREADS) {
+            const uint32_t key = K.ckey[q];
+            g += key > Tk;
+            e += key == Tk;
+        }
+        g = __reduce_add_sync(~0u, g);
+        e = __reduce_add_sync(~0u, e);
+        if (lane_id() == 0 && (g | e)) {
+            atomicAdd(&K.cnt[0], g);
+            atomicAdd(&K.cnt[1], e);
+        }
     }
     if (c == 0 && tid == 0 && p.hint_tag != 0) {
         if (hb != NO_KEY) {
@@ -666,6 +736,7 @@ small_kernel(const __grid_constant__ SmallParams p) {
         K.sh = sh;
         K.armed = armed == sk_arm(seq) ? 1u : 0u;
         K.cnt[0] = K.cnt[1] = 0;
+        K.lcnt = 0;
         if (c == 0) {
             ctrl->path_small = SK_PATH_TAG;
             ctrl->sk_tag = (uint32_t)K.tag;
