@@ -525,8 +525,9 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
     }
     for (int i = tid; i < FS_WARPS * 32; i += FS_THREADS) F.wbm[i] = 0u;
     __syncthreads();
-    // the k-th key's bin b1, and the 2k-th key's bin for the next call's hint
-    fs_find2(F.hist, k, 2 * k, F);
+    // the k-th key's bin b1, and the (3k/2)-th key's bin for the next call's
+    // hint
+    fs_find2(F.hist, k, k + k / 2, F);
     mark_phase(ctrl, 1);
     const FindResult f1 = F.fr1;
     const uint32_t total = F.total;
@@ -548,8 +549,8 @@ flat_select_kernel(const __grid_constant__ FlatParams p) {
     const uint32_t lmask = (1u << sh) - 1u;
     uint32_t hint_T0 = 0;
     if (c == 0 && tid == 0 && p.hint) {
-        // next call: the threshold where this call's 2k-th key lies (or this
-        // one's T0 if there were fewer than 2k candidates), with the widest
+        // next call: the threshold where this call's (3k/2)-th key lies (or
+        // this one's T0 if there were fewer candidates), with the widest
         // relative digits (4,095 bins of 2^12 keys: up to four times T0 in
         // value), so that a k-th key that grows from step to step stays in
         // range
