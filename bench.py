@@ -259,10 +259,10 @@ def l2_note(flush: bool, input_bytes: int) -> str:
 
 def hbm_bar(wl, frac):
     """The 60%-of-HBM bar set for the Top-k + EF compress of n >= 25.6M
-    elements, judged on the whole call; other workloads are not held to it."""
+    elements, measured on the whole call; other workloads are not held to it."""
     if isinstance(wl, (FlatCompress, BatchedCompress)) and wl.n >= datagen.RESNET50_N:
-        return {"judged_on": "whole call (hbm_frac_whole_step): setup, streaming pass "
-                             "and select", "bar": 0.60, "met": bool(frac >= 0.60)}
+        return {"measured_on": "whole call (hbm_frac_whole_step): setup, streaming pass "
+                               "and select", "bar": 0.60, "met": bool(frac >= 0.60)}
     return {"applies": False,
             "why": "the bar is set for the Top-k + EF compress of n >= 25.6M elements"}
 
