@@ -16,6 +16,7 @@ constexpr int MG_THREADS = 512;
 constexpr int MG_PER_THREAD = 4;
 constexpr int MG_D = MG_THREADS * MG_PER_THREAD;   // merged positions per block
 constexpr int MZ_THREADS = 512;
+constexpr int MZ_LOADS = 12;                       // index loads in flight per thread
 
 struct MergeSetupParams {
     const int32_t* in_idx;
@@ -45,14 +46,18 @@ struct MergeSetupParams {
 __global__ void __launch_bounds__(MZ_THREADS)
 merge_setup_kernel(const MergeSetupParams p) {
     const int b = blockIdx.x, tid = threadIdx.x;
-    // the first round may be scheduled now (it waits for this grid); this
-    // grid waits for the kernel before it on the stream
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // this grid waits for the kernel before it on the stream.  The first
+    // round may be scheduled once every block of this grid has finished its
+    // work (each triggers at its end), not from the start: scheduled while
+    // these blocks still hold the SMs, its clusters are placed piecemeal
+    // and no longer fit in one wave (measured on the 32-worker tournament:
+    // 149 against 124 us per call)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((uint32_t)b < p.validate_blocks) {
         // a contiguous range of the P * k_in entries per block; each thread's
         // position inside its row is carried along (no division per entry),
-        // and four entries and their successors are loaded at once
+        // and MZ_LOADS entries and their successors are loaded at once (one
+        // round trip for the 32-worker tournament's 11 entries per thread)
         const int64_t tot = (int64_t)p.P * p.k_in;
         const int64_t per = (tot + p.validate_blocks - 1) / p.validate_blocks;
         const int64_t e0 = min((int64_t)b * per, tot), e1 = min(e0 + per, tot);
@@ -62,11 +67,11 @@ merge_setup_kernel(const MergeSetupParams p) {
         const int64_t step = (int64_t)blockDim.x;
         const int64_t jstep = step % p.k_in;
         while (e < e1) {
-            int32_t v[4], w[4];
-            bool last[4];
+            int32_t v[MZ_LOADS], w[MZ_LOADS];
+            bool last[MZ_LOADS];
             int64_t ee = e, jj = j;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < MZ_LOADS; ++u) {
                 last[u] = jj + 1 >= p.k_in;      // no successor in the row
                 v[u] = ee < e1 ? p.in_idx[ee] : 0;
                 w[u] = (ee < e1 && !last[u]) ? p.in_idx[ee + 1] : 0;
@@ -75,7 +80,7 @@ merge_setup_kernel(const MergeSetupParams p) {
                 if (jj >= p.k_in) jj -= p.k_in;
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < MZ_LOADS; ++u) {
                 if (e + u * step >= e1) break;
                 if (v[u] < 0 || (int64_t)v[u] >= p.n) bad = true;
                 if (!last[u] && w[u] <= v[u]) bad = true;
@@ -85,6 +90,7 @@ merge_setup_kernel(const MergeSetupParams p) {
         }
         const int any = __syncthreads_or(bad);
         if (tid == 0) p.bad_words[b] = any ? 1u : 0u;
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         return;
     }
     const int zb = b - (int)p.validate_blocks;
@@ -113,6 +119,7 @@ merge_setup_kernel(const MergeSetupParams p) {
     for (uint64_t i = (uint64_t)zb * blockDim.x + tid; i < p.zero_vec4;
          i += (uint64_t)nz * blockDim.x)
         p.zero_ptr[i] = z;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 struct MergeRoundParams {

@@ -39,7 +39,18 @@ struct McCfg {
     static constexpr int QMAX = PT * MC_THREADS;                      // positions per CTA
     static constexpr int STAGE = 4 * (QMAX + 1);                      // staging words
     static constexpr int GCAP = STAGE - QMAX - 4;                     // gathered list capacity
+    // digit-1 bins whose cluster sum one CTA owns (a multiple of 4; the last
+    // CTA's slice ends at D1_BINS)
+    static constexpr int SB = ((D1_BINS + CL - 1) / CL + 3) / 4 * 4;
+    // first step of a binary search over the cluster ranks 0 .. CL - 1
+    static constexpr int ST0 = CL > 8 ? 8 : CL > 4 ? 4 : CL > 2 ? 2 : 1;
 };
+
+// Merged positions of a pair that a cluster of CL CTAs holds.
+template <int CL>
+constexpr int64_t mc_pair_cap() {
+    return (int64_t)CL * McCfg<CL>::QMAX;
+}
 
 // Relative digit 1 (rounds after the first): bin 0 holds the keys below the
 // pair's floor L (sums at common indices can fall there), bins 1 .. 2046 the
@@ -93,6 +104,7 @@ struct McFixed {
     uint32_t loff[17];                                // list offsets by cluster rank
     uint32_t lcnt[16];                                // list lengths by cluster rank
     __align__(16) uint32_t hslice[D1_BINS / 8];       // this CTA's slice of the summed h1
+                                                      // (McCfg<CL>::SB <= D1_BINS / 8 bins)
     uint32_t live_tot;
     uint32_t E, pre_above;
     FindResult fr;
@@ -129,9 +141,11 @@ __device__ __forceinline__ void cluster_find(cg::cluster_group& cl, McFixed& S, 
 }
 
 template <int CL>
-__global__ void __launch_bounds__(MC_THREADS, (CL >= 16 ? 2 : 1))
+__global__ void __launch_bounds__(MC_THREADS, (CL >= 12 ? 2 : 1))
 merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     using C = McCfg<CL>;
+    static_assert(CL >= 8 && CL <= 16, "clusters of 8 to 16 CTAs");
+    static_assert(C::SB * CL >= D1_BINS && C::SB <= D1_BINS / 8, "digit-1 slices");
     constexpr int PT = C::PT;
     constexpr int QMAX = C::QMAX;
     extern __shared__ __align__(16) unsigned char mc_smem[];
@@ -185,7 +199,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     for (int i = tid; i < D1_BINS; i += blockDim.x) S.h1[i] = 0;
     for (int i = tid; i < D2_BINS; i += blockDim.x) S.h2[i] = 0;
     for (int i = tid; i < D3_BINS; i += blockDim.x) S.h3[i] = 0;
-    for (int i = tid; i < D1_BINS / CL; i += blockDim.x) S.hslice[i] = 0;
+    for (int i = tid; i < C::SB; i += blockDim.x) S.hslice[i] = 0;
     __syncthreads();
     if (stamp) p.ctrl->t_phase[1] = global_ns();
     const int64_t i0 = S.part[0], i1 = max(S.part[1], i0);
@@ -295,7 +309,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         rel = false;
         cl.sync();
         for (int i = tid; i < D1_BINS; i += blockDim.x) S.h1[i] = 0;
-        for (int i = tid; i < D1_BINS / CL; i += blockDim.x) S.hslice[i] = 0;
+        for (int i = tid; i < C::SB; i += blockDim.x) S.hslice[i] = 0;
         __syncthreads();
 #pragma unroll
         for (int u = 0; u < PT; ++u)
@@ -305,9 +319,9 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     if (stamp) p.ctrl->t_phase[4] = global_ns();
 
     // live entries of the pair (warp 0, lane r reads rank r), and this CTA's
-    // slice of the summed digit-1 histogram: bins [cr*SB, cr*SB + SB) over
-    // all CTAs, one 16-byte remote load per thread
-    constexpr int SB = D1_BINS / CL;
+    // slice of the summed digit-1 histogram: bins [cr*SB, cr*SB + SB) (up to
+    // D1_BINS) over all CTAs, one 16-byte remote load per thread
+    constexpr int SB = C::SB;
     if (tid < 32) {
         const uint32_t lv = tid < CL ? *cl.map_shared_rank(&S.live, tid) : 0u;
         const uint32_t lt = warp_sum(lv);
@@ -315,6 +329,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
     }
     for (int t = tid; t < (SB / 4) * CL; t += blockDim.x) {
         const int r = t / (SB / 4), j = t - r * (SB / 4);
+        if (cr * SB + 4 * j >= D1_BINS) continue;
         const uint4 v = *reinterpret_cast<const uint4*>(cl.map_shared_rank(S.h1 + cr * SB + 4 * j, r));
         atomicAdd(&S.hslice[4 * j + 0], v.x);
         atomicAdd(&S.hslice[4 * j + 1], v.y);
@@ -418,7 +433,7 @@ merge_cluster_kernel(const __grid_constant__ MergeClusterParams p) {
         for (uint32_t u = tid; u < E / 4; u += blockDim.x) {
             int r = 0;
 #pragma unroll
-            for (int st = CL / 2; st >= 1; st >>= 1)
+            for (int st = C::ST0; st >= 1; st >>= 1)
                 if (r + st < CL && S.loff[r + st] <= 4 * u) r += st;
             const uint32_t i = 4 * u - S.loff[r];          // first entry of the load
             uint4 v = *reinterpret_cast<const uint4*>(cl.map_shared_rank(mylist + i, r));

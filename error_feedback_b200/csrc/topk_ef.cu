@@ -648,14 +648,21 @@ size_t threshold_workspace(int64_t n) {
     return compress_layout(n, plans).total;
 }
 
-// The cluster merge kernel: clusters of 16 CTAs (a non-portable size) or of
-// 8, whichever the device can hold; found once per device.
+// The cluster merge kernel: one cluster of CL CTAs per pair, CL = 16, 14 or
+// 12 at two CTAs per SM (sizes above 8 are non-portable) or 8 at one.  How
+// many clusters of each size the device holds at once is found once per
+// device.
+constexpr int MC_SIZES[4] = {16, 14, 12, 8};
+struct McFit {
+    int active[4];              // resident clusters of MC_SIZES[i] CTAs (0: cannot run)
+};
 std::mutex g_mc_mu;
-int g_mc_fit[64];               // 0 not yet probed; else 1 + (16 fits) + 2 * (8 fits)
+bool g_mc_probed[64];
+McFit g_mc_fit[64];
 
 template <int CL>
-cudaError_t mc_config(bool* fits) {
-    *fits = false;
+cudaError_t mc_config(int* active) {
+    *active = 0;
     cudaError_t e = cudaFuncSetAttribute(merge_cluster_kernel<CL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)mc_smem_bytes<CL>());
@@ -683,34 +690,56 @@ cudaError_t mc_config(bool* fits) {
         cudaGetLastError();
         return cudaSuccess;
     }
-    *fits = clusters > 0;
+    *active = clusters > 0 ? clusters : 0;
     return cudaSuccess;
 }
 
-// Cluster sizes this device can hold: bit 0 for 16, bit 1 for 8 (0: the
-// cluster kernel cannot run).
-int merge_cluster_sizes(int* mask_out) {
+int merge_cluster_fit(McFit* out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= 64) return TOPK_EF_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lk(g_mc_mu);
-    if (g_mc_fit[dev] == 0) {
-        bool f16 = false, f8 = false;
-        if ((e = mc_config<16>(&f16)) != cudaSuccess) return cuda_fail(e);
-        if ((e = mc_config<8>(&f8)) != cudaSuccess) return cuda_fail(e);
-        g_mc_fit[dev] = 1 + (f16 ? 1 : 0) + (f8 ? 2 : 0);
+    if (!g_mc_probed[dev]) {
+        McFit f;
+        if ((e = mc_config<16>(&f.active[0])) != cudaSuccess) return cuda_fail(e);
+        if ((e = mc_config<14>(&f.active[1])) != cudaSuccess) return cuda_fail(e);
+        if ((e = mc_config<12>(&f.active[2])) != cudaSuccess) return cuda_fail(e);
+        if ((e = mc_config<8>(&f.active[3])) != cudaSuccess) return cuda_fail(e);
+        g_mc_fit[dev] = f;
+        g_mc_probed[dev] = true;
     }
-    *mask_out = g_mc_fit[dev] - 1;
+    *out = g_mc_fit[dev];
     return TOPK_EF_OK;
 }
 
-// Cluster size of a round: 16 CTAs per pair wherever the device holds such
-// a cluster, else 8.  (Rounds with more pairs than 16-CTA clusters fit one
-// per SM still run faster with 16-CTA clusters at two CTAs per SM than with
-// 8-CTA clusters at one: measured 43.7 against 53.5 us for the first round
-// of the 32-worker tournament.)
-int round_cluster(int mask) { return (mask & 1) ? 16 : 8; }
+int64_t mc_cap(int i) {
+    switch (i) {
+        case 0: return mc_pair_cap<16>();
+        case 1: return mc_pair_cap<14>();
+        case 2: return mc_pair_cap<12>();
+        default: return mc_pair_cap<8>();
+    }
+}
+
+// Cluster size of a round of np pairs whose merged lists hold up to mcap
+// positions (0: no size can run it).  16 CTAs per pair when the device holds
+// all np such clusters at once.  Else the largest of 14 and 12 of which it
+// does: fewer CTAs per pair, but one wave of clusters instead of two.  Else
+// 16 in several waves (they still ran faster than one wave of 8-CTA clusters
+// at one CTA per SM: 43.7 against 53.5 us for the first round of the
+// 32-worker tournament), or 8 where the device holds no larger cluster.
+// `forced` (a test flag: an index into MC_SIZES, or -1) picks a size
+// wherever that size can run.
+int round_cluster(const McFit& f, int32_t np, int64_t mcap, int forced) {
+    auto fits = [&](int i) { return f.active[i] > 0 && mcap <= mc_cap(i); };
+    if (forced >= 0 && forced < 4 && fits(forced)) return MC_SIZES[forced];
+    if (fits(0) && np <= f.active[0]) return 16;
+    for (int i = 1; i <= 2; ++i)
+        if (fits(i) && np <= f.active[i]) return MC_SIZES[i];
+    if (fits(0)) return 16;
+    return fits(3) ? 8 : 0;
+}
 
 template <int CL>
 cudaError_t launch_mc(int32_t np, cudaStream_t st, const MergeClusterParams& cp) {
@@ -733,7 +762,12 @@ cudaError_t launch_mc(int32_t np, cudaStream_t st, const MergeClusterParams& cp)
 
 cudaError_t launch_merge_cluster(int cl, int32_t np, cudaStream_t st,
                                  const MergeClusterParams& cp) {
-    return cl == 16 ? launch_mc<16>(np, st, cp) : launch_mc<8>(np, st, cp);
+    switch (cl) {
+        case 16: return launch_mc<16>(np, st, cp);
+        case 14: return launch_mc<14>(np, st, cp);
+        case 12: return launch_mc<12>(np, st, cp);
+        default: return launch_mc<8>(np, st, cp);
+    }
 }
 
 bool bad_fp32_ptr(const void* p) { return ((uintptr_t)p & 3u) != 0; }
@@ -1079,13 +1113,18 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
     uint32_t* m_idx = reinterpret_cast<uint32_t*>(w + L.m_idx);
     float* m_val = reinterpret_cast<float*>(w + L.m_val);
     const bool single = (P == 1 || k_in == 0);
-    // one cluster kernel per round when every round's merged lists fit
+    // one cluster kernel per round when a cluster size holds every round
     bool cluster_path = !single;
     for (int r = 0; r < L.rounds; ++r)
         cluster_path = cluster_path && L.mcap[r] <= MC_PAIR_MAX;
-    int mc_mask = 0;
-    if (cluster_path && (rc = merge_cluster_sizes(&mc_mask)) != TOPK_EF_OK) return rc;
-    cluster_path = cluster_path && mc_mask != 0;
+    McFit fit;
+    if (cluster_path && (rc = merge_cluster_fit(&fit)) != TOPK_EF_OK) return rc;
+    const int forced_cl = ((g_test_flags.load() >> 3) & 7) - 1;
+    std::vector<int> cls(L.rounds, 0);
+    for (int r = 0; cluster_path && r < L.rounds; ++r) {
+        cls[r] = round_cluster(fit, L.np[r], L.mcap[r], forced_cl);
+        cluster_path = cls[r] != 0;
+    }
     const uint32_t kernels =
         single ? 2u : (uint32_t)(cluster_path ? 1 + L.rounds : 1 + 2 * L.rounds);
 
@@ -1186,7 +1225,7 @@ int gtopk_merge(const int32_t* in_idx, const float* in_val, int32_t P, int64_t k
             cp.n_bad = r == 0 ? (int32_t)L.vblocks : 0;
             cp.ctrl = ctrl;
             trace_before(st, "merge_cluster_kernel");
-            e = launch_merge_cluster(round_cluster(mc_mask), L.np[r], st, cp);
+            e = launch_merge_cluster(cls[r], L.np[r], st, cp);
             trace_after(st);
             if (e != cudaSuccess) return cuda_fail(e);
         }

@@ -350,7 +350,10 @@ int topk_ef_phase_times(const void* ws, void* stream, int64_t* ns);
  * large tensors and so also ends in the fallback); bit 2 makes the grid-wide
  * exchange of a single-tensor compress call wait for one block more than
  * the grid has, so that its bounded wait runs out (after about a second) and
- * the call records TOPK_EF_ERR_DEVICE_TIMEOUT, with undefined outputs.  0
+ * the call records TOPK_EF_ERR_DEVICE_TIMEOUT, with undefined outputs; bits
+ * 3..5, when 1, 2, 3 or 4, make the rounds of gtopk_merge that one thread-block
+ * cluster per pair can hold use clusters of 16, 14, 12 or 8 CTAs wherever
+ * that size can run (else the size is chosen per round as usual).  0
  * restores normal behaviour.  Returns the previous flags.  The flags are
  * process-wide state read by every call in the process (the library's only
  * state outside the caller's workspace besides the tracing record and the

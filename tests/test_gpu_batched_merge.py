@@ -200,3 +200,23 @@ def test_merge_relative_digit_falls_back(case):
     idx = np.stack([I, J, I, J]).astype(np.int32)
     val = np.stack(vals).astype(np.float32)
     run_merge(idx, val, k, n, ws=_mws(4, k, k))
+
+
+@pytest.mark.parametrize("size", [16, 14, 12, 8])
+@pytest.mark.parametrize("P,k_in,k,n", [
+    (32, 25_557, 25_557, datagen.RESNET50_N),
+    (13, 3_001, 2_500, 200_000),
+])
+def test_merge_cluster_sizes(size, P, k_in, k, n):
+    """Every cluster size of the cluster kernel (one pair per cluster of
+    16, 14, 12 or 8 CTAs; 16, 14 and 12 divide digit 1's 2,048 bins into
+    slices of 128, 148 and 172, the last slice shorter), forced through the
+    test flag for every round."""
+    idx, val = datagen.gtopk_sets(P=P, k=k_in, n=n, step=size)
+    ws = _mws(P, k_in, k)
+    old = ef.topk_ef_set_test_flags({16: 1, 14: 2, 12: 3, 8: 4}[size] << 3)
+    try:
+        run_merge(idx, val, k, n, ws=ws)
+    finally:
+        ef.topk_ef_set_test_flags(old)
+    assert ef.topk_ef_path_info(ws)["kernels"] == 1 + (P - 1).bit_length()
