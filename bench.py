@@ -679,11 +679,12 @@ def run_ours(args):
     # timed region: K steps; inputs larger than L2 run back to back, smaller
     # ones get an L2 flush before each step (outside the timed intervals).
     # Only the dominant kernel is bracketed by events, and only a few of its
-    # launches spread over the region (one per ten, at most TRACE_BRACKETS):
+    # launches spread over the region (one per twenty, at least one, at most
+    # TRACE_BRACKETS):
     # events between two launches stop the second from starting early, so
     # every bracket slows the step it falls in.
     dom_launches = sum(1 for name, _ in trace_all if name == wl.dominant) * args.steps // nt
-    brackets = min(TRACE_BRACKETS, max(1, dom_launches // 10))
+    brackets = min(TRACE_BRACKETS, max(1, dom_launches // 20))
     every = max(1, -(-dom_launches // brackets))
     ef.topk_ef_trace_enable(True, only=wl.dominant, every=every)
     barrier()
