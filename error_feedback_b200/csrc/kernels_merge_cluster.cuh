@@ -5,16 +5,19 @@
 // one thread-block cluster of CL CTAs:
 //   1. CTA c merges its share of the pair's merged list (merge path) into
 //      registers and builds the histogram of the first radix digit (key
-//      bits 30..20);
+//      bits 30..20 in the first round; after it, bins of 2^13 keys above the
+//      lower of the two sets' lowest keys);
 //   2. the digit histograms are summed over the cluster through distributed
-//      shared memory, which gives the bin b1 of the k-th key;
+//      shared memory (each CTA sums a slice, then reads every slice), which
+//      gives the bin b1 of the k-th key;
 //   3. every CTA lists its entries in bin b1 (with its rank in the cluster)
 //      and counts those above it; every CTA then gathers all the lists and
 //      finds, locally, the k-th key T, the tie quota q and its own output
 //      offset (the counts above b1 of the CTAs before it plus their listed
 //      entries above / equal to T);
 //   4. every CTA writes its share of the top k in index order.
-// Three cluster barriers, no grid barrier.  A bin b1 with more entries than
+// Four cluster barriers (the last keeps each CTA's shared memory alive for
+// the others' reads), no grid barrier.  A bin b1 with more entries than
 // the gather space resolves the remaining digits by two more summed
 // histogram passes and exchanges exact counts instead.  Used when a round's
 // merged lists fit (CL * QMAX positions per pair); larger rounds take the
