@@ -5,8 +5,14 @@
 //                                 (flat_select_kernel for a single tensor,
 //                                 select_kernel<CompressSrc> for a bucket);
 //                                 a single small tensor: small_kernel alone
-//   gtopk_merge:                  merge_setup_kernel -> (merge_round_kernel ->
-//                                 select_kernel) per tournament round
+//   gtopk_merge:                  merge_setup_kernel -> merge_cluster_kernel per
+//                                 tournament round (one thread-block cluster per
+//                                 pair), or (merge_round_kernel -> select_kernel)
+//                                 per round when a pair's merged list exceeds
+//                                 what a cluster holds
+//   topk_ef_threshold:            setup_kernel -> stream_kernel -> threshold_kernel
+//   gtopk_residual_return:        return_kernel
+//   topk_allgather_sum:           ag_bounds_kernel -> ag_sum_kernel
 //
 // Every launch goes to the caller's stream; nothing is allocated and nothing
 // is synchronised except by the two status read-back calls.
